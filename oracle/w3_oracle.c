@@ -1,0 +1,201 @@
+/*
+ * w3_oracle.c -- plain, slow CPU oracle for the W3A16 group-128 format.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path (the CUDA library
+ * and its Python binding) may include, link, load or call this file.  Only the
+ * tests, the smoke check and the CPU-baseline leg of the benchmark use it.  It
+ * shares no code with the CUDA kernels: it is written at the level of single
+ * bits and single multiply-adds so that a reader can check it against the
+ * format definition by eye.
+ *
+ * What it follows (all from the GSQ model card "Llama-3.1-70B-Instruct-3Bit-GSQ",
+ * section "Storage layout (why the HF UI shows I32 + BF16)" and the
+ * quantization_config block under it):
+ *   - a weight of shape [N, K] (out_features, in_features) is stored as uint3
+ *     codes with exact-width packing: no code is padded into a wider field, so
+ *     a row of K codes takes K*3/32 int32 words ("8192 x 3 / 32 = 768");
+ *   - one bf16 scale per group of 128 consecutive weights along K, shape
+ *     [N, K/128] ("8192 / 128 = 64"), weight_scale_type "group",
+ *     weight_scale_group_size 128;
+ *   - symmetric, has_zero_point false: a weight is (signed level) x scale;
+ *   - section "Quantization details": the GSQ codebook is the 5-level integer
+ *     set {-2,-1,0,1,+2} times the group scale.
+ *
+ * Readings where the card is silent (each is also listed with the design notes):
+ *   - bit order: one LSB-first bitstream per row.  Code k of row n occupies
+ *     stream bits 3k, 3k+1, 3k+2 (bit 0 of the code first), and stream bit b
+ *     is bit (b mod 32) of word floor(b/32) of that row.  Equivalently, the 3
+ *     words of each 32-code block, read as one little-endian 96-bit integer,
+ *     equal sum_j c_j * 8^j.
+ *   - signed level: q = c - 4 for every code c in 0..7, so the GSQ levels
+ *     -2..2 are the codes 2..6.
+ *   - int32 container: a raw 32-bit pattern (handled here as uint32_t).
+ *   - the product y = x * W^T (nn.Linear convention), W[n,k] = q[n,k]*s[n,k/128].
+ *
+ * Precision: the fp32 dequantized weight q*s is exact (|q| <= 4 is a 3-bit
+ * integer and a bf16 scale has 8 significant bits, so the product has at most
+ * 11), and the matrix product is accumulated in fp64 in plain k order.
+ *
+ * Every function returns 0 on success and -1 on an invalid argument.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_GROUP 128
+
+/* Words of packed storage per row: K codes x 3 bits / 32 bits per word. */
+int64_t oracle_words_per_row(int64_t K) {
+    if (K <= 0 || (K * 3) % 32 != 0) return -1;
+    return K * 3 / 32;
+}
+
+/* Scale groups per row: one bf16 scale per 128 weights along K. */
+int64_t oracle_groups_per_row(int64_t K) {
+    if (K <= 0 || K % ORACLE_GROUP != 0) return -1;
+    return K / ORACLE_GROUP;
+}
+
+/* bf16 is the upper half of an IEEE binary32: widen by appending 16 zero bits. */
+static float bf16_bits_to_float(uint16_t h) {
+    uint32_t u = ((uint32_t)h) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* Read one bit of row `row` (a pointer to its first word) at stream position b. */
+static unsigned stream_bit(const uint32_t *row, int64_t b) {
+    return (unsigned)((row[b / 32] >> (b % 32)) & 1u);
+}
+
+/* The 3-bit code c[n,k], assembled bit by bit from the row's bitstream. */
+static unsigned code_at(const uint32_t *row, int64_t k) {
+    unsigned c = 0;
+    for (int i = 0; i < 3; ++i)
+        c |= stream_bit(row, 3 * k + i) << i;
+    return c;
+}
+
+/* codes: [N,K] bytes, each 0..7.  packed: [N, K*3/32] words, fully written. */
+int oracle_pack(const uint8_t *codes, uint32_t *packed, int64_t N, int64_t K) {
+    int64_t W = oracle_words_per_row(K);
+    if (!codes || !packed || N < 0 || W < 0) return -1;
+    for (int64_t n = 0; n < N; ++n) {
+        uint32_t *row = packed + n * W;
+        for (int64_t w = 0; w < W; ++w) row[w] = 0;
+        for (int64_t k = 0; k < K; ++k) {
+            unsigned c = codes[n * K + k];
+            if (c > 7) return -1;
+            for (int i = 0; i < 3; ++i) {
+                int64_t b = 3 * k + i;
+                uint32_t bit = (c >> i) & 1u;
+                row[b / 32] |= bit << (b % 32);
+            }
+        }
+    }
+    return 0;
+}
+
+/* packed: [N, K*3/32] words.  codes: [N,K] bytes, each written with 0..7. */
+int oracle_unpack(const uint32_t *packed, uint8_t *codes, int64_t N, int64_t K) {
+    int64_t W = oracle_words_per_row(K);
+    if (!codes || !packed || N < 0 || W < 0) return -1;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k)
+            codes[n * K + k] = (uint8_t)code_at(packed + n * W, k);
+    return 0;
+}
+
+/* w[n,k] = (c[n,k] - 4) * s[n, k/128] in fp32 (exact).  scales: bf16 bits [N, K/128]. */
+int oracle_dequant_f32(const uint32_t *packed, const uint16_t *scales, float *w,
+                       int64_t N, int64_t K) {
+    int64_t W = oracle_words_per_row(K), G = oracle_groups_per_row(K);
+    if (!packed || !scales || !w || N < 0 || W < 0 || G < 0) return -1;
+    for (int64_t n = 0; n < N; ++n) {
+        const uint32_t *row = packed + n * W;
+        for (int64_t k = 0; k < K; ++k) {
+            int q = (int)code_at(row, k) - 4;
+            float s = bf16_bits_to_float(scales[n * G + k / ORACLE_GROUP]);
+            w[n * K + k] = (float)q * s;
+        }
+    }
+    return 0;
+}
+
+/* One output element: sum over k of x[m,k] * W[n,k], fp64, k ascending. */
+static double dot_row(const uint16_t *x, const float *wrow, int64_t m, int64_t K) {
+    double acc = 0.0;
+    for (int64_t k = 0; k < K; ++k)
+        acc += (double)bf16_bits_to_float(x[m * K + k]) * (double)wrow[k];
+    return acc;
+}
+
+/* Dequantize row n of W into wrow (K floats). */
+static void dequant_row(const uint32_t *packed, const uint16_t *scales, int64_t n,
+                        int64_t K, float *wrow) {
+    int64_t W = K * 3 / 32, G = K / ORACLE_GROUP;
+    const uint32_t *row = packed + n * W;
+    for (int64_t k = 0; k < K; ++k) {
+        int q = (int)code_at(row, k) - 4;
+        wrow[k] = (float)q * bf16_bits_to_float(scales[n * G + k / ORACLE_GROUP]);
+    }
+}
+
+/*
+ * y[m,n] = sum_k x[m,k] * W[n,k]   (y = x W^T), y in fp64, row-major [M,N].
+ * x: bf16 bits [M,K]; packed: [N,K*3/32]; scales: bf16 bits [N,K/128].
+ */
+int oracle_gemm_f64(const uint16_t *x, const uint32_t *packed, const uint16_t *scales,
+                    double *y, int64_t M, int64_t N, int64_t K) {
+    if (!x || !packed || !scales || !y || M < 0 || N < 0) return -1;
+    if (oracle_words_per_row(K) < 0 || oracle_groups_per_row(K) < 0) return -1;
+    float *wrow = (float *)malloc((size_t)K * sizeof(float));
+    if (!wrow) return -1;
+    for (int64_t n = 0; n < N; ++n) {
+        dequant_row(packed, scales, n, K, wrow);
+        for (int64_t m = 0; m < M; ++m)
+            y[m * N + n] = dot_row(x, wrow, m, K);
+    }
+    free(wrow);
+    return 0;
+}
+
+/*
+ * The same product for a list of `count` single entries (ms[i], ns[i]), for
+ * checking sampled outputs of shapes too large for the full triple loop.
+ */
+int oracle_gemm_f64_entries(const uint16_t *x, const uint32_t *packed,
+                            const uint16_t *scales, int64_t M, int64_t N, int64_t K,
+                            const int64_t *ms, const int64_t *ns, int64_t count,
+                            double *out) {
+    if (!x || !packed || !scales || !ms || !ns || !out || count < 0) return -1;
+    if (oracle_words_per_row(K) < 0 || oracle_groups_per_row(K) < 0) return -1;
+    float *wrow = (float *)malloc((size_t)K * sizeof(float));
+    if (!wrow) return -1;
+    for (int64_t i = 0; i < count; ++i) {
+        if (ms[i] < 0 || ms[i] >= M || ns[i] < 0 || ns[i] >= N) { free(wrow); return -1; }
+        dequant_row(packed, scales, ns[i], K, wrow);
+        out[i] = dot_row(x, wrow, ms[i], K);
+    }
+    free(wrow);
+    return 0;
+}
+
+/* ||W[n,:]||_2 of the dequantized row, in fp64 (used by the output tolerance). */
+int oracle_weight_row_norms(const uint32_t *packed, const uint16_t *scales,
+                            int64_t N, int64_t K, double *out) {
+    if (!packed || !scales || !out || N < 0) return -1;
+    if (oracle_words_per_row(K) < 0 || oracle_groups_per_row(K) < 0) return -1;
+    float *wrow = (float *)malloc((size_t)K * sizeof(float));
+    if (!wrow) return -1;
+    for (int64_t n = 0; n < N; ++n) {
+        dequant_row(packed, scales, n, K, wrow);
+        double ss = 0.0;
+        for (int64_t k = 0; k < K; ++k) ss += (double)wrow[k] * (double)wrow[k];
+        out[n] = sqrt(ss);
+    }
+    free(wrow);
+    return 0;
+}
