@@ -1,0 +1,402 @@
+#!/usr/bin/env python3
+"""Benchmark of the W3A16 group-128 decode path on B200.
+
+Workload (one "step"): the Llama-3.1-70B gate_proj shape N=28672, K=8192 with
+uint3 codes uniform over 0..7 and lognormal(-4, 0.5) bf16 group scales, run as
+three w3a16_gemm calls with batch M = 1, 4 and 16 (x ~ N(0,1) bf16).  Each call
+reads a different copy of the weights; five copies (459 MB) rotate, so every
+call streams its 91.8 MB of weights from HBM rather than from the 126 MB L2.
+
+Reported: effective HBM GB/s = algorithmic bytes / time, where the algorithmic
+bytes of one call are N*K*3/8 (packed) + N*K/128*2 (scales) + M*K*2 (x) +
+M*N*2 (y).  `roofline` is the dominant kernel's per-launch figure against the
+measured HBM copy bandwidth.  `e2e` is the same metric through the Python API
+with x copied from pinned host memory and y copied back every call.
+`cpu_baseline` times the CPU oracle on a bounded sample of the same step.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+Under torchrun each rank runs an independent replica (the path does not shard);
+value = bytes of all ranks / the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "W3A16 g128 µs/call and effective HBM GB/s (% of B200 peak) at Llama-70B shapes"
+UNIT = "GB/s"
+N_ROWS, K_COLS = 28672, 8192
+BATCHES = (1, 4, 16)
+ROTATE = 5
+WORKLOAD = "Llama-3.1-70B gate_proj N=28672 K=8192, W3A16 g128 decode batch M=1,4,16"
+FALLBACK_HBM_GBS = 6650.0
+DECODE_SOURCES = ("w3a16_gemv_b200/csrc/decode_gemv.cuh", "w3a16_gemv_b200/csrc/common.cuh")
+
+
+def algorithmic_bytes(M: int, N: int, K: int) -> int:
+    return N * K * 3 // 8 + N * (K // 128) * 2 + M * K * 2 + M * N * 2
+
+
+def step_bytes() -> int:
+    return sum(algorithmic_bytes(m, N_ROWS, K_COLS) for m in BATCHES)
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs: STREAM-style copy, burst)"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback (6.65 TB/s earlier measurement on this pool)"
+
+
+def sources_sha() -> str:
+    h = hashlib.sha256()
+    for rel in DECODE_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel_m: int):
+    """DRAM bytes per launch from the committed ncu summary, if it matches the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if d.get("source_sha") != sources_sha():
+        return None
+    v = d.get("dram_bytes_per_launch", {}).get(f"M{kernel_m}")
+    return float(v) if v is not None else None
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML in a background thread."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.002):
+        self.samples = []  # (t, sm_mhz, reasons)
+        self.period = period_s
+        self._stop = threading.Event()
+        self.ok = False
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:  # NVML missing: clocks are reported as unavailable
+            self.max_mhz = None
+
+    def _sample(self):
+        nv = self.nv
+        mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+        try:
+            r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except AttributeError:
+            r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+        self.samples.append((time.perf_counter(), mhz, r))
+
+    def _run(self):
+        while not self._stop.is_set():
+            self._sample()
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+            self._sample()
+
+    def summary(self, t0: float, t1: float):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        if not inside:  # timed region shorter than the sampling period: nearest samples
+            inside = sorted(self.samples, key=lambda s: min(abs(s[0] - t0), abs(s[0] - t1)))[:2]
+        reasons = 0
+        for s in inside:
+            reasons |= s[2]
+        names = sorted(n for bit, n in self.REASONS.items() if reasons & bit and bit != 0x1)
+        return {"sm_mhz": float(statistics.median(s[1] for s in inside)), "sm_max_mhz": float(self.max_mhz),
+                "reasons": names, "samples": len(inside)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+# --------------------------------------------------------------------------------------
+# CPU oracle (the reported baseline and the reference arm)
+# --------------------------------------------------------------------------------------
+
+def oracle_step_sample(budget_s: float):
+    """Time the oracle on the first rows of the step until `budget_s` of CPU work is spent.
+
+    Returns (GB/s in the metric's unit, seconds, rows, description)."""
+    import oracle
+    from w3a16_gemv_b200.inputs import make_problem
+
+    orc = oracle.get()
+    rows_per_chunk = 256
+    p = make_problem(max(BATCHES), rows_per_chunk, K_COLS, "uniform8", "lognormal", "normal", seed=0)
+    packed = orc.pack(p.codes)
+    done_rows, spent, nbytes = 0, 0.0, 0
+    while spent < budget_s and done_rows < N_ROWS:
+        t0 = time.perf_counter()
+        for m in BATCHES:
+            orc.gemm_f64(p.x_bf16[:m], packed, p.scales_bf16)
+        spent += time.perf_counter() - t0
+        done_rows += rows_per_chunk
+    # bytes of the sampled rows in the metric's accounting (weights + the x/y share)
+    frac = done_rows / N_ROWS
+    nbytes = step_bytes() * frac
+    desc = (f"oracle_gemm_f64 (plain C, one thread) for M=1,4,16 over K=8192 on {done_rows} weight rows "
+            f"(a 256-row slice of the seeded workload, repeated; {frac:.2%} of one step's rows), "
+            f"GB/s = the step's algorithmic bytes scaled by rows / CPU seconds")
+    return nbytes / spent / 1e9, spent, done_rows, desc
+
+
+def run_reference(args):
+    world, rank, _ = dist_setup()
+    if rank != 0:
+        return 0
+    per_step = []
+    # keep the whole run within a few minutes whatever --steps/--warmup are
+    budget = max(0.2, min(args.ref_budget, 150.0 / (args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_step_sample(min(0.5, budget))
+    desc = None
+    for _ in range(args.steps):
+        gbs, spent, rows, desc = oracle_step_sample(budget)
+        per_step.append((gbs, spent))
+    value = statistics.median(g for g, _ in per_step)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": statistics.median(1e3 * s for _, s in per_step), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "sample": desc},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------------------
+# GPU arm
+# --------------------------------------------------------------------------------------
+
+def run_gpu(args):
+    import torch
+
+    from w3a16_gemv_b200 import build as wbuild
+    from w3a16_gemv_b200 import w3_check_device_error, w3_pack, w3a16_gemm
+    from w3a16_gemv_b200.inputs import make_problem
+
+    world, rank, local = dist_setup()
+    if world > 1:
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if not os.path.exists(wbuild.LIB):
+        wbuild.build()
+
+    # ---- inputs: seeded, drawn on the host, packed on the device by w3_pack ----
+    p = make_problem(max(BATCHES), N_ROWS, K_COLS, "uniform8", "lognormal", "normal", seed=0)
+    codes_d = torch.from_numpy(p.codes).to(dev)
+    packed0 = w3_pack(codes_d)
+    del codes_d
+    scales0 = torch.from_numpy(p.scales_bf16.view(np.int16)).view(torch.bfloat16).to(dev)
+    packs = [packed0] + [packed0.clone() for _ in range(ROTATE - 1)]
+    scales = [scales0] + [scales0.clone() for _ in range(ROTATE - 1)]
+    x_all = torch.from_numpy(p.x_bf16.view(np.int16)).view(torch.bfloat16).to(dev)
+    xs = {m: x_all[:m].contiguous() for m in BATCHES}
+    ys = {m: torch.empty((m, N_ROWS), dtype=torch.bfloat16, device=dev) for m in BATCHES}
+    torch.cuda.synchronize()
+
+    calls_per_step = len(BATCHES)
+    stream = torch.cuda.current_stream()
+
+    def one_step(i, ev=None):
+        for j, m in enumerate(BATCHES):
+            c = (i * calls_per_step + j) % ROTATE
+            if ev is not None:
+                ev[j][0].record(stream)
+            w3a16_gemm(xs[m], packs[c], scales[c], out=ys[m])
+            if ev is not None:
+                ev[j][1].record(stream)
+
+    for i in range(args.warmup):
+        one_step(i)
+    torch.cuda.synchronize()
+    w3_check_device_error()
+
+    # ---- timed region: K steps, barrier + synchronize on both sides ----
+    events = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
+               for _ in BATCHES] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.02)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    w0 = time.perf_counter()
+    t_start.record(stream)
+    for i in range(args.steps):
+        one_step(args.warmup + i, events[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    w1 = time.perf_counter()
+    if world > 1:
+        torch.distributed.barrier()
+    sampler.stop()
+    w3_check_device_error()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    per_call_ms = {m: [events[i][j][0].elapsed_time(events[i][j][1]) for i in range(args.steps)]
+                   for j, m in enumerate(BATCHES)}
+
+    if world > 1:
+        t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+
+    total_bytes = step_bytes() * args.steps * world
+    value = total_bytes / (elapsed_ms * 1e-3) / 1e9
+    ms_per_step = elapsed_ms / args.steps
+
+    # ---- roofline of the dominant kernel (largest share of the step) ----
+    peak, peak_src = measured_peak()
+    calls = []
+    for m in BATCHES:
+        us = 1e3 * statistics.mean(per_call_ms[m])
+        b = algorithmic_bytes(m, N_ROWS, K_COLS)
+        calls.append({"M": m, "us_mean": us, "us_median": 1e3 * statistics.median(per_call_ms[m]),
+                      "GB/s": b / (us * 1e-6) / 1e9, "TFLOP/s": 2.0 * m * N_ROWS * K_COLS / (us * 1e-6) / 1e12,
+                      "frac_of_peak": b / (us * 1e-6) / 1e9 / peak, "share": 0.0})
+    tot = sum(c["us_mean"] for c in calls)
+    for c in calls:
+        c["share"] = c["us_mean"] / tot
+    dom = max(calls, key=lambda c: c["us_mean"])
+    traffic = recorded_traffic(dom["M"])
+    roofline = {"bound": "hbm", "achieved": dom["GB/s"], "peak": peak, "unit": "GB/s",
+                "frac": dom["GB/s"] / peak, "traffic": traffic,
+                "kernel": f"w3::decode::decode_kernel<{1 if dom['M'] <= 8 else 2}> (M={dom['M']})",
+                "algorithmic_bytes_per_launch": algorithmic_bytes(dom["M"], N_ROWS, K_COLS),
+                "peak_source": peak_src}
+
+    # ---- end to end through the public API with host buffers ----
+    x_host = {m: torch.empty((m, K_COLS), dtype=torch.bfloat16).pin_memory() for m in BATCHES}
+    for m in BATCHES:
+        x_host[m].copy_(xs[m].cpu())
+    y_host = {m: torch.empty((m, N_ROWS), dtype=torch.bfloat16).pin_memory() for m in BATCHES}
+    xd = {m: torch.empty_like(xs[m]) for m in BATCHES}
+    e2e_steps = max(1, min(args.steps, 200))
+
+    def e2e_step(i):
+        for j, m in enumerate(BATCHES):
+            c = (i * calls_per_step + j) % ROTATE
+            xd[m].copy_(x_host[m], non_blocking=True)
+            w3a16_gemm(xd[m], packs[c], scales[c], out=ys[m])
+            y_host[m].copy_(ys[m], non_blocking=True)
+        stream.synchronize()
+
+    for i in range(3):
+        e2e_step(i)
+    if world > 1:
+        torch.distributed.barrier()
+    e0 = time.perf_counter()
+    for i in range(e2e_steps):
+        e2e_step(i)
+    e_ms = (time.perf_counter() - e0) * 1e3
+    if world > 1:
+        t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e_ms = float(t.item())
+    e2e = {"value": step_bytes() * e2e_steps * world / (e_ms * 1e-3) / 1e9, "unit": UNIT,
+           "h2d_bytes_per_step": sum(m * K_COLS * 2 for m in BATCHES),
+           "d2h_bytes_per_step": sum(m * N_ROWS * 2 for m in BATCHES),
+           "steps": e2e_steps, "ms_per_step": e_ms / e2e_steps}
+
+    clocks = sampler.summary(w0, w1)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "M": list(BATCHES), "N": N_ROWS, "K": K_COLS,
+                   "codes": "uniform 0..7", "scales": "bf16 lognormal(-4, 0.5)", "x": "bf16 N(0,1)",
+                   "l2": f"inputs larger than L2: {ROTATE} rotating weight copies "
+                         f"({ROTATE * algorithmic_bytes(0, N_ROWS, K_COLS) / 1e6:.0f} MB > 126 MB)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "step_bytes": step_bytes()},
+        "us_per_call": {f"M{c['M']}": c["us_mean"] for c in calls},
+        "calls": calls,
+        "roofline": roofline,
+        "e2e": e2e,
+        "gpu_launches": args.steps * calls_per_step,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        gbs, spent, rows, desc = oracle_step_sample(args.cpu_budget)
+        line["cpu_baseline"] = {"value": gbs, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc,
+                                "seconds": spent}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of CPU oracle work for cpu_baseline")
+    ap.add_argument("--ref-budget", type=float, default=3.0, help="seconds of oracle work per reference step")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,130 @@
+/*
+ * w3a16.h -- C ABI of libw3a16.so: W3A16 group-128 fused dequantize-and-multiply
+ * for NVIDIA B200 (sm_100a).
+ *
+ * Format (GSQ model card "Llama-3.1-70B-Instruct-3Bit-GSQ", section "Storage
+ * layout (why the HF UI shows I32 + BF16)" and its quantization_config block):
+ *   - a linear layer's weight W has shape [N, K] = [out_features, in_features];
+ *   - it is stored as uint3 codes with exact-width packing, 32 codes in 3
+ *     int32 words, so `packed` is [N, 3K/32] int32, row-major ("8192 x 3 / 32
+ *     = 768" in the card's gate_proj example);
+ *   - one bf16 scale per group of 128 consecutive weights along K, so
+ *     `scales` is [N, K/128] bf16, row-major ("8192 / 128 = 64");
+ *   - symmetric, no zero point: W[n,k] = (c[n,k] - 4) * scales[n, k/128].
+ *     The GSQ codebook (section "Quantization details") uses the levels
+ *     -2..+2, i.e. codes 2..6; codes 0, 1 and 7 (levels -4, -3, +3) are valid too.
+ *
+ * Bit order (the card does not print one; this library fixes it): each row is
+ * one LSB-first bitstream.  Code k occupies stream bits 3k..3k+2, bit 0 of
+ * the code first, and stream bit b is bit (b mod 32) of word b/32 of the row.
+ * Read as one little-endian 96-bit integer, the 3 words of every 32-code block
+ * equal sum_j c_j * 8^j.  Codes 10 and 21 of each block straddle a word boundary.
+ *
+ * Conventions for every entry point:
+ *   - all array pointers are DEVICE pointers (cudaMalloc'd or torch CUDA
+ *     tensors) on the current device; the caller owns every buffer and the
+ *     library allocates no device memory;
+ *   - bf16 values are passed as their 16-bit patterns (uint16_t);
+ *   - every array pointer must be 16-byte aligned (W3_ERR_ALIGN otherwise);
+ *   - calls only enqueue work on `stream` (NULL = the legacy default stream)
+ *     and return immediately; results are visible after the stream is
+ *     synchronised;
+ *   - the return value is the status; no call aborts, throws or exits;
+ *   - arguments are checked on the host before anything is launched; a
+ *     failing check returns an error and enqueues nothing;
+ *   - a device-side wait that runs out of time (a hardware or driver fault,
+ *     never expected) records W3_ERR_TIMEOUT in a per-device flag that
+ *     w3_check_device_error() reports.
+ */
+#ifndef W3A16_H
+#define W3A16_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* The same object as cudaStream_t; declared here so this header needs no CUDA headers. */
+typedef struct CUstream_st *w3_stream_t;
+
+typedef enum w3_status {
+    W3_OK = 0,
+    W3_ERR_NULL = 1,        /* a required pointer is NULL */
+    W3_ERR_SHAPE = 2,       /* a size is out of range: M, N < 1, K < 128, K % 128 != 0, or too large */
+    W3_ERR_ALIGN = 3,       /* an array pointer is not 16-byte aligned */
+    W3_ERR_CUDA = 4,        /* the CUDA runtime reported an error (launch, device query) */
+    W3_ERR_UNSUPPORTED = 5, /* the current device is not sm_100 (B200/GB200) */
+    W3_ERR_TIMEOUT = 6,     /* a bounded device-side wait gave up (see w3_check_device_error) */
+    W3_ERR_ALIAS = 7        /* the output overlaps an input */
+} w3_status;
+
+/* A short English description of a status; never NULL. */
+const char *w3_status_string(w3_status status);
+
+/* Version of this ABI (incremented on any incompatible change). */
+int32_t w3_abi_version(void);
+
+/* int32 words per packed row, 3K/32; -1 if K is not a positive multiple of 128. */
+int64_t w3_packed_words_per_row(int64_t K);
+
+/* bf16 scales per row, K/128; -1 if K is not a positive multiple of 128. */
+int64_t w3_groups_per_row(int64_t K);
+
+/*
+ * w3_pack -- codes [N,K] uint8 (values 0..7; the upper 5 bits of each byte are
+ * ignored) -> packed [N, 3K/32] int32 in the bit order above.
+ * Storage layout from the card's "Storage layout" section.  Every output word
+ * is written.  Errors: W3_ERR_NULL, W3_ERR_SHAPE (N < 1, K not a positive
+ * multiple of 128), W3_ERR_ALIGN, W3_ERR_ALIAS (codes and packed overlap),
+ * W3_ERR_UNSUPPORTED, W3_ERR_CUDA.
+ */
+w3_status w3_pack(const uint8_t *codes, int32_t *packed, int64_t N, int64_t K, w3_stream_t stream);
+
+/*
+ * w3_unpack -- packed [N, 3K/32] int32 -> codes [N,K] uint8 (each 0..7).
+ * The inverse of w3_pack (same section of the card).  Same errors as w3_pack.
+ */
+w3_status w3_unpack(const int32_t *packed, uint8_t *codes, int64_t N, int64_t K, w3_stream_t stream);
+
+/*
+ * w3_dequant_f32 -- w[n,k] = (c[n,k] - 4) * scales[n, k/128] as fp32 [N,K].
+ * The symmetric group-wise dequantization of the card's quantization_config
+ * (weight_scale_type "group", weight_scale_group_size 128, has_zero_point
+ * false).  The product is exact in fp32.  Meant for checking and debugging;
+ * the product entry point below never materialises W.  Same errors as w3_pack.
+ */
+w3_status w3_dequant_f32(const int32_t *packed, const uint16_t *scales, float *w,
+                         int64_t N, int64_t K, w3_stream_t stream);
+
+/*
+ * w3a16_gemm -- y = x * W^T (the nn.Linear product of the card's quantized
+ * Linear layers), with W dequantized on the fly and never written to memory.
+ *   x      [M,K] bf16, row-major
+ *   packed [N, 3K/32] int32, scales [N, K/128] bf16 (the format above)
+ *   y      [M,N] bf16, row-major; every element is written
+ * Arithmetic: fp32 accumulation; the result is rounded once to bf16 (nearest
+ * even).  For M <= 16 the weight enters the products exactly (q and the
+ * scale are applied in fp32); for M > 16 each weight is first rounded to
+ * bf16(q*s) and fed to the tensor cores.  Repeated calls with the same
+ * arguments give bit-identical y (no floating-point atomics).
+ * Errors: W3_ERR_NULL, W3_ERR_SHAPE (M, N < 1; K < 128 or K % 128 != 0;
+ * M*K, N*K or M*N above 2^40), W3_ERR_ALIGN, W3_ERR_ALIAS (y overlaps x,
+ * packed or scales), W3_ERR_UNSUPPORTED, W3_ERR_CUDA.
+ */
+w3_status w3a16_gemm(const uint16_t *x, const int32_t *packed, const uint16_t *scales, uint16_t *y,
+                     int64_t M, int64_t N, int64_t K, w3_stream_t stream);
+
+/*
+ * w3_check_device_error -- synchronise `stream`, then report and clear the
+ * current device's error flag: W3_OK, or W3_ERR_TIMEOUT if a kernel of this
+ * library gave up a bounded wait since the last check.  W3_ERR_CUDA if the
+ * synchronisation itself fails.
+ */
+w3_status w3_check_device_error(w3_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W3A16_H */

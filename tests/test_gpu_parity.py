@@ -1,0 +1,161 @@
+"""GPU parity: the CUDA library, called through its C ABI, against the CPU oracle.
+
+* pack / unpack / fp32 dequant: bit-exact.
+* y = x W^T: every checked element within |y - y_ref| <= 1e-2*||x_m||*||w_n||/sqrt(K) + 1e-3
+  of the fp64 oracle.
+Small shapes are checked in full (several tiles, ragged edges, every decode
+batch size); the full-size workloads are checked on sampled outputs computed
+one by one by the oracle, in the same launch configuration the benchmark times.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_helpers import assert_within_bound, bound, device_problem, from_dev_bf16
+from w3a16_gemv_b200 import build, w3_check_device_error, w3_dequant_f32, w3_pack, w3_unpack, w3a16_gemm
+from w3a16_gemv_b200.inputs import make_problem, workloads
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    build.build()
+    assert torch.cuda.is_available()
+
+
+# (M, N, K, codes, scales, x): odd and ragged sizes, one group, odd group counts,
+# every M the decode path handles, and batches above 16.
+SMALL = [
+    (1, 1, 128, "uniform8", "lognormal", "normal"),
+    (1, 17, 128, "uniform8", "lognormal", "normal"),
+    (2, 64, 384, "gsq_uniform", "absnormal", "normal"),
+    (3, 100, 1152, "uniform8", "lognormal", "normal_outliers"),
+    (4, 250, 640, "gsq_5level", "absnormal", "normal"),
+    (5, 64, 4096, "uniform8", "lognormal", "normal"),
+    (7, 129, 256, "uniform8", "lognormal", "normal"),
+    (8, 333, 2048, "uniform8", "absnormal", "normal_outliers"),
+    (9, 77, 768, "gsq_uniform", "lognormal", "normal"),
+    (12, 300, 1024, "uniform8", "lognormal", "normal"),
+    (16, 129, 256, "uniform8", "lognormal", "normal"),
+    (16, 1000, 8192, "uniform8", "lognormal", "normal"),
+    (1, 2000, 128, "uniform8", "lognormal", "normal"),
+    (1, 64, 28672, "gsq_5level", "absnormal", "normal_outliers"),
+    (17, 50, 512, "uniform8", "lognormal", "normal"),
+    (40, 96, 1280, "uniform8", "lognormal", "normal"),
+]
+
+
+def _id(c):
+    return f"M{c[0]}_N{c[1]}_K{c[2]}_{c[3]}"
+
+
+@pytest.mark.parametrize("case", SMALL, ids=[_id(c) for c in SMALL])
+def test_small_shapes_full_parity(orc, case):
+    M, N, K, cd, sd, xd = case
+    p = make_problem(M, N, K, cd, sd, xd, seed=11)
+    x, codes, scales = device_problem(p)
+    packed = w3_pack(codes)
+    ref_packed = orc.pack(p.codes)
+    assert np.array_equal(packed.cpu().numpy().view(np.uint32), ref_packed)
+    assert np.array_equal(w3_unpack(packed, K).cpu().numpy(), p.codes)
+    w = w3_dequant_f32(packed, scales, K).cpu().numpy()
+    assert np.array_equal(w.view(np.uint32), orc.dequant_f32(ref_packed, p.scales_bf16, K).view(np.uint32))
+    y = w3a16_gemm(x, packed, scales)
+    w3_check_device_error()
+    ref = orc.gemm_f64(p.x_bf16, ref_packed, p.scales_bf16)
+    tol = bound(p.x_bf16, orc.weight_row_norms(ref_packed, p.scales_bf16, K), K)
+    assert_within_bound(from_dev_bf16(y), ref, tol, _id(case))
+
+
+def test_all_levels_exact_dequant_and_gsq_levels(orc):
+    # every code value at every block position, and the GSQ levels -2..2 for codes 2..6
+    N, K = 8, 256
+    codes = (np.arange(N * K).reshape(N, K) % 8).astype(np.uint8)
+    codes[1] = np.arange(K) // 32 % 8
+    p = make_problem(1, N, K, "uniform8", "lognormal", "normal", seed=12)
+    _, _, scales = device_problem(p)
+    packed = w3_pack(torch.from_numpy(codes).cuda())
+    assert np.array_equal(packed.cpu().numpy().view(np.uint32), orc.pack(codes))
+    w = w3_dequant_f32(packed, scales, K).cpu().numpy()
+    s = oracle.bf16_to_f64(p.scales_bf16)
+    want = (codes.astype(np.float64) - 4.0) * np.repeat(s, 128, axis=1)
+    assert np.array_equal(w.astype(np.float64), want)
+
+
+def test_deterministic_repeated_calls():
+    p = make_problem(4, 3000, 4096, seed=13)
+    x, codes, scales = device_problem(p)
+    packed = w3_pack(codes)
+    ys = [from_dev_bf16(w3a16_gemm(x, packed, scales)) for _ in range(3)]
+    assert all(np.array_equal(ys[0], y) for y in ys[1:])
+
+
+def test_batch_rows_match_single_row_calls(orc):
+    """Row m of an M=16 call against the M=1 call on that row: both within the bound;
+    bit-identity is reported (not required: the split of K may differ with M)."""
+    p = make_problem(16, 512, 2048, seed=14)
+    x, codes, scales = device_problem(p)
+    packed = w3_pack(codes)
+    yb = from_dev_bf16(w3a16_gemm(x, packed, scales))
+    ref = orc.gemm_f64(p.x_bf16, orc.pack(p.codes), p.scales_bf16)
+    tol = bound(p.x_bf16, orc.weight_row_norms(orc.pack(p.codes), p.scales_bf16, 2048), 2048)
+    same = 0
+    for m in range(16):
+        y1 = from_dev_bf16(w3a16_gemm(x[m:m + 1].contiguous(), packed, scales))
+        assert_within_bound(y1, ref[m:m + 1], tol[m:m + 1], f"row {m}")
+        same += int(np.array_equal(y1[0], yb[m]))
+    print(f"batch-invariance: {same}/16 rows bit-identical between M=1 and M=16")
+
+
+def test_position_probe(orc):
+    # x = e_k picks column k of W: the result is one dequantized weight, rounded once
+    N, K = 40, 256
+    p = make_problem(16, N, K, seed=15)
+    _, codes, scales = device_problem(p)
+    packed = w3_pack(codes)
+    w = orc.dequant_f32(orc.pack(p.codes), p.scales_bf16, K)
+    for k0 in range(0, K, 16):
+        eye = np.zeros((16, K), dtype=np.float32)
+        eye[np.arange(16), k0 + np.arange(16)] = 1.0
+        x = torch.from_numpy(eye).to(torch.bfloat16).cuda()
+        y = oracle.bf16_to_f64(from_dev_bf16(w3a16_gemm(x, packed, scales)))
+        want = w[:, k0:k0 + 16].T.astype(np.float64)
+        assert np.all(np.abs(y - want) <= 2.0 ** -8 * np.abs(want) + 1e-30), k0
+
+
+def _sampled_check(orc, name, n_samples=1024, seed=0):
+    wl = workloads()[name]
+    p = wl.problem()
+    x, codes, scales = device_problem(p)
+    packed = w3_pack(codes)
+    ref_packed = orc.pack(p.codes)
+    assert np.array_equal(packed.cpu().numpy().view(np.uint32), ref_packed), "pack differs from the oracle"
+    del codes
+    y = from_dev_bf16(w3a16_gemm(x, packed, scales))
+    w3_check_device_error()
+    rng = np.random.Generator(np.random.PCG64(seed))
+    ms = rng.integers(0, wl.M, n_samples)
+    ns = rng.integers(0, wl.N, n_samples)
+    # always include the corners and the last row/column
+    ms = np.concatenate([ms, [0, wl.M - 1, 0, wl.M - 1]])
+    ns = np.concatenate([ns, [0, 0, wl.N - 1, wl.N - 1]])
+    ref = orc.gemm_f64_entries(p.x_bf16, ref_packed, p.scales_bf16, ms, ns)
+    norms = orc.weight_row_norms(ref_packed[ns], p.scales_bf16[ns], wl.K)
+    xf = oracle.bf16_to_f64(p.x_bf16[ms])
+    tol = 1e-2 * np.sqrt(np.sum(xf * xf, axis=1)) * norms / np.sqrt(wl.K) + 1e-3
+    worst = assert_within_bound(y[ms, ns][None, :], ref[None, :], tol[None, :], name)
+    print(f"{name}: worst |err|/bound = {worst:.3g} over {ms.size} sampled outputs")
+
+
+FULL = [n for n in workloads() if not n.startswith("prefill")]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_sampled(orc, name):
+    _sampled_check(orc, name)
+
+
+def test_prefill_full_size_sampled(orc):
+    _sampled_check(orc, "prefill_2048x28672x8192", n_samples=4096)

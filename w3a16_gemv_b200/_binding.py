@@ -1,0 +1,174 @@
+"""ctypes binding of libw3a16.so: argument marshalling only.
+
+Each function here has the name of the C entry point it calls (see
+``include/w3a16.h``), takes torch CUDA tensors, checks dtypes and shapes,
+allocates outputs with torch when none are given, and passes raw pointers and
+torch's current CUDA stream to the library.  No arithmetic of the format or of
+the product happens in Python, and there is no fallback: if the library is
+missing or the device is not a B200, the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libw3a16.so")
+
+W3_OK = 0
+STATUS_NAMES = {
+    0: "W3_OK",
+    1: "W3_ERR_NULL",
+    2: "W3_ERR_SHAPE",
+    3: "W3_ERR_ALIGN",
+    4: "W3_ERR_CUDA",
+    5: "W3_ERR_UNSUPPORTED",
+    6: "W3_ERR_TIMEOUT",
+    7: "W3_ERR_ALIAS",
+}
+
+# (name, restype, argtypes) of every entry point declared in include/w3a16.h
+_P, _I64 = ctypes.c_void_p, ctypes.c_int64
+SIGNATURES = [
+    ("w3_status_string", ctypes.c_char_p, [ctypes.c_int]),
+    ("w3_abi_version", ctypes.c_int32, []),
+    ("w3_packed_words_per_row", _I64, [_I64]),
+    ("w3_groups_per_row", _I64, [_I64]),
+    ("w3_pack", ctypes.c_int, [_P, _P, _I64, _I64, _P]),
+    ("w3_unpack", ctypes.c_int, [_P, _P, _I64, _I64, _P]),
+    ("w3_dequant_f32", ctypes.c_int, [_P, _P, _P, _I64, _I64, _P]),
+    ("w3a16_gemm", ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P]),
+    ("w3_check_device_error", ctypes.c_int, [_P]),
+]
+
+_lock = threading.Lock()
+_lib: ctypes.CDLL | None = None
+
+
+class W3Error(RuntimeError):
+    """A non-zero w3_status returned by the library."""
+
+    def __init__(self, status: int, what: str):
+        self.status = status
+        name = STATUS_NAMES.get(status, str(status))
+        super().__init__(f"{what}: {name} ({status_string(status)})")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library with its signatures declared.  Raises if it was not built."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(
+                    f"{LIB_PATH} is missing: build it with `python -m w3a16_gemv_b200.build` "
+                    "(there is no fallback implementation)")
+            handle = ctypes.CDLL(LIB_PATH)
+            for name, res, args in SIGNATURES:
+                f = getattr(handle, name)
+                f.restype = res
+                f.argtypes = args
+            _lib = handle
+        return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().w3_status_string(int(status)).decode()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _check(status: int, what: str) -> None:
+    if status != W3_OK:
+        raise W3Error(status, what)
+
+
+def _need(t: torch.Tensor, dtype: torch.dtype, name: str) -> None:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def w3_packed_words_per_row(K: int) -> int:
+    return int(lib().w3_packed_words_per_row(K))
+
+
+def w3_groups_per_row(K: int) -> int:
+    return int(lib().w3_groups_per_row(K))
+
+
+def w3_pack(codes: torch.Tensor, packed: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """codes uint8 [N,K] (0..7) -> packed int32 [N, 3K/32]."""
+    _need(codes, torch.uint8, "codes")
+    N, K = codes.shape
+    if packed is None:
+        packed = torch.empty((N, max(w3_packed_words_per_row(K), 1)), dtype=torch.int32, device=codes.device)
+    _need(packed, torch.int32, "packed")
+    _check(lib().w3_pack(codes.data_ptr(), packed.data_ptr(), N, K, _stream(stream)), "w3_pack")
+    return packed
+
+
+def w3_unpack(packed: torch.Tensor, K: int, codes: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """packed int32 [N, 3K/32] -> codes uint8 [N,K]."""
+    _need(packed, torch.int32, "packed")
+    N = packed.shape[0]
+    if packed.shape[1] != w3_packed_words_per_row(K):
+        raise ValueError("packed width does not match K")
+    if codes is None:
+        codes = torch.empty((N, K), dtype=torch.uint8, device=packed.device)
+    _need(codes, torch.uint8, "codes")
+    _check(lib().w3_unpack(packed.data_ptr(), codes.data_ptr(), N, K, _stream(stream)), "w3_unpack")
+    return codes
+
+
+def w3_dequant_f32(packed: torch.Tensor, scales: torch.Tensor, K: int, out: torch.Tensor | None = None,
+                   stream=None) -> torch.Tensor:
+    """W[n,k] = (c-4) * scales[n,k//128] as float32 [N,K]."""
+    _need(packed, torch.int32, "packed")
+    _need(scales, torch.bfloat16, "scales")
+    N = packed.shape[0]
+    if packed.shape[1] != w3_packed_words_per_row(K) or tuple(scales.shape) != (N, w3_groups_per_row(K)):
+        raise ValueError("packed/scales shapes do not match N, K")
+    if out is None:
+        out = torch.empty((N, K), dtype=torch.float32, device=packed.device)
+    _need(out, torch.float32, "out")
+    _check(lib().w3_dequant_f32(packed.data_ptr(), scales.data_ptr(), out.data_ptr(), N, K, _stream(stream)),
+           "w3_dequant_f32")
+    return out
+
+
+def w3a16_gemm(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, out: torch.Tensor | None = None,
+               stream=None) -> torch.Tensor:
+    """y = x W^T, x bf16 [M,K], packed int32 [N,3K/32], scales bf16 [N,K/128] -> y bf16 [M,N]."""
+    _need(x, torch.bfloat16, "x")
+    _need(packed, torch.int32, "packed")
+    _need(scales, torch.bfloat16, "scales")
+    M, K = x.shape
+    N = packed.shape[0]
+    if packed.shape[1] != w3_packed_words_per_row(K) or tuple(scales.shape) != (N, w3_groups_per_row(K)):
+        raise ValueError("packed/scales shapes do not match x's K")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _need(out, torch.bfloat16, "out")
+    if tuple(out.shape) != (M, N):
+        raise ValueError("out must be [M, N]")
+    _check(lib().w3a16_gemm(x.data_ptr(), packed.data_ptr(), scales.data_ptr(), out.data_ptr(), M, N, K,
+                            _stream(stream)), "w3a16_gemm")
+    return out
+
+
+def w3_check_device_error(stream=None) -> None:
+    """Synchronise the stream and raise W3Error if a kernel recorded a timeout."""
+    _check(lib().w3_check_device_error(_stream(stream)), "w3_check_device_error")

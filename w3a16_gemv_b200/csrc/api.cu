@@ -1,0 +1,264 @@
+// api.cu -- the extern "C" entry points of libw3a16.so (declared in include/w3a16.h).
+//
+// Host side only: argument checks, per-device set-up, kernel selection and
+// launch.  All arithmetic runs in the kernels included below (one translation
+// unit, so the device error flag needs no relocatable device code).
+#include <atomic>
+#include <cstdint>
+#include <mutex>
+
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include "../../include/w3a16.h"
+#include "common.cuh"
+#include "decode_gemv.cuh"
+#include "format_kernels.cuh"
+
+#ifndef W3_DECODE_TMA2D
+#define W3_DECODE_TMA2D 1
+#endif
+
+namespace w3 {
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int64_t kMaxElems = int64_t(1) << 40;
+constexpr int64_t kMaxDim = int64_t(1) << 30;
+
+struct DeviceState {
+    std::once_flag once;
+    w3_status status = W3_OK;
+    int num_sms = 0;
+};
+DeviceState g_dev[kMaxDevices];
+
+// Once per device: check that it is an sm_100 part and raise the kernels'
+// dynamic shared-memory limits.
+w3_status device_setup(int *num_sms) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return W3_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return W3_ERR_UNSUPPORTED;
+    DeviceState &st = g_dev[dev];
+    std::call_once(st.once, [&] {
+        int major = 0, minor = 0, sms = 0, optin = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) {
+            st.status = W3_ERR_CUDA;
+            return;
+        }
+        if (major != 10 || minor != 0) {
+            st.status = W3_ERR_UNSUPPORTED;
+            return;
+        }
+        st.num_sms = sms;
+        const void *kernels[] = {
+            reinterpret_cast<const void *>(decode::decode_kernel<1>),
+            reinterpret_cast<const void *>(decode::decode_kernel<2>),
+            reinterpret_cast<const void *>(decode::decode_kernel<4>),
+            reinterpret_cast<const void *>(decode::decode_kernel<8>),
+            reinterpret_cast<const void *>(decode::decode_kernel<16>),
+        };
+        for (const void *k : kernels) {
+            if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, optin) != cudaSuccess) {
+                st.status = W3_ERR_CUDA;
+                return;
+            }
+        }
+        st.status = W3_OK;
+    });
+    *num_sms = st.num_sms;
+    return st.status;
+}
+
+// cuTensorMapEncodeTiled from the driver, fetched once through the runtime.
+PFN_cuTensorMapEncodeTiled tensor_map_encoder() {
+    static std::once_flag once;
+    static PFN_cuTensorMapEncodeTiled fn = nullptr;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled>(p);
+    });
+    return fn;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlaps(const void *a, int64_t abytes, const void *b, int64_t bbytes) {
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+    return a0 < b0 + static_cast<uintptr_t>(bbytes) && b0 < a0 + static_cast<uintptr_t>(abytes);
+}
+
+w3_status check_nk(int64_t N, int64_t K) {
+    if (N < 1 || K < kGroup || K % kGroup != 0) return W3_ERR_SHAPE;
+    if (N > kMaxDim || K > kMaxDim || N * K > kMaxElems) return W3_ERR_SHAPE;
+    return W3_OK;
+}
+
+w3_status launch_status() {
+    return cudaGetLastError() == cudaSuccess ? W3_OK : W3_ERR_CUDA;
+}
+
+w3_status launch_decode(const uint16_t *x, const int32_t *packed, const uint16_t *scales, uint16_t *y, int M,
+                        int N, int K, int num_sms, cudaStream_t stream) {
+    const decode::LaunchPlan P = decode::plan(M, N, K, num_sms);
+    decode::Params prm;
+    prm.x = x;
+    prm.packed = reinterpret_cast<const uint32_t *>(packed);
+    prm.scales = scales;
+    prm.y = y;
+    prm.M = M;
+    prm.N = N;
+    prm.K = K;
+    prm.groups_per_cta = P.groups_per_cta;
+    prm.gchunk = P.gchunk;
+    // one tiled TMA copy per stage when the box fits inside the matrix, else per-row bulk copies
+    prm.use_tma2d = 0;
+    const int64_t words = static_cast<int64_t>(K) * 3 / 32;
+    if (W3_DECODE_TMA2D && N >= decode::kRowsPerWarp && words >= decode::kRowPitchWords) {
+        PFN_cuTensorMapEncodeTiled enc = tensor_map_encoder();
+        if (!enc) return W3_ERR_CUDA;
+        cuuint64_t dims[2] = {static_cast<cuuint64_t>(words), static_cast<cuuint64_t>(N)};
+        cuuint64_t strides[1] = {static_cast<cuuint64_t>(words * 4)};
+        cuuint32_t box[2] = {decode::kRowPitchWords, decode::kRowsPerWarp};
+        cuuint32_t estr[2] = {1, 1};
+        if (enc(&prm.tmap, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<int32_t *>(packed), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return W3_ERR_CUDA;
+        prm.use_tma2d = 1;
+    }
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = P.grid;
+    cfg.blockDim = dim3(decode::kWarps * 32, 1, 1);
+    cfg.dynamicSmemBytes = P.smem_bytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    if (P.cluster > 1) {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 1;
+        attr[0].val.clusterDim.y = P.cluster;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    cudaError_t e;
+    switch (P.mt) {
+        case 1: e = cudaLaunchKernelEx(&cfg, decode::decode_kernel<1>, prm); break;
+        case 2: e = cudaLaunchKernelEx(&cfg, decode::decode_kernel<2>, prm); break;
+        case 4: e = cudaLaunchKernelEx(&cfg, decode::decode_kernel<4>, prm); break;
+        case 8: e = cudaLaunchKernelEx(&cfg, decode::decode_kernel<8>, prm); break;
+        default: e = cudaLaunchKernelEx(&cfg, decode::decode_kernel<16>, prm); break;
+    }
+    return e == cudaSuccess ? W3_OK : W3_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace w3
+
+using namespace w3;
+
+extern "C" {
+
+const char *w3_status_string(w3_status s) {
+    switch (s) {
+        case W3_OK: return "ok";
+        case W3_ERR_NULL: return "a required pointer is NULL";
+        case W3_ERR_SHAPE: return "a size is out of range (M, N >= 1; K a positive multiple of 128)";
+        case W3_ERR_ALIGN: return "an array pointer is not 16-byte aligned";
+        case W3_ERR_CUDA: return "the CUDA runtime reported an error";
+        case W3_ERR_UNSUPPORTED: return "the current device is not an sm_100 (B200) GPU";
+        case W3_ERR_TIMEOUT: return "a device-side wait timed out";
+        case W3_ERR_ALIAS: return "the output overlaps an input";
+    }
+    return "unknown status";
+}
+
+int32_t w3_abi_version(void) { return 1; }
+
+int64_t w3_packed_words_per_row(int64_t K) {
+    return (K >= kGroup && K % kGroup == 0) ? K * 3 / 32 : -1;
+}
+
+int64_t w3_groups_per_row(int64_t K) { return (K >= kGroup && K % kGroup == 0) ? K / kGroup : -1; }
+
+w3_status w3_pack(const uint8_t *codes, int32_t *packed, int64_t N, int64_t K, w3_stream_t stream) {
+    if (!codes || !packed) return W3_ERR_NULL;
+    if (w3_status s = check_nk(N, K)) return s;
+    if (!aligned16(codes) || !aligned16(packed)) return W3_ERR_ALIGN;
+    if (overlaps(codes, N * K, packed, N * K * 3 / 8)) return W3_ERR_ALIAS;
+    int sms;
+    if (w3_status s = device_setup(&sms)) return s;
+    const int64_t nblocks = N * K / 32;
+    pack_kernel<<<grid_for(nblocks, 256), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        codes, reinterpret_cast<uint32_t *>(packed), nblocks);
+    return launch_status();
+}
+
+w3_status w3_unpack(const int32_t *packed, uint8_t *codes, int64_t N, int64_t K, w3_stream_t stream) {
+    if (!codes || !packed) return W3_ERR_NULL;
+    if (w3_status s = check_nk(N, K)) return s;
+    if (!aligned16(codes) || !aligned16(packed)) return W3_ERR_ALIGN;
+    if (overlaps(codes, N * K, packed, N * K * 3 / 8)) return W3_ERR_ALIAS;
+    int sms;
+    if (w3_status s = device_setup(&sms)) return s;
+    const int64_t nblocks = N * K / 32;
+    unpack_kernel<<<grid_for(nblocks, 256), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        reinterpret_cast<const uint32_t *>(packed), codes, nblocks);
+    return launch_status();
+}
+
+w3_status w3_dequant_f32(const int32_t *packed, const uint16_t *scales, float *w, int64_t N, int64_t K,
+                         w3_stream_t stream) {
+    if (!packed || !scales || !w) return W3_ERR_NULL;
+    if (w3_status s = check_nk(N, K)) return s;
+    if (!aligned16(packed) || !aligned16(scales) || !aligned16(w)) return W3_ERR_ALIGN;
+    if (overlaps(w, N * K * 4, packed, N * K * 3 / 8) || overlaps(w, N * K * 4, scales, N * (K / kGroup) * 2))
+        return W3_ERR_ALIAS;
+    int sms;
+    if (w3_status s = device_setup(&sms)) return s;
+    const int64_t nblocks = N * K / 32;
+    dequant_f32_kernel<<<grid_for(nblocks, 256), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        reinterpret_cast<const uint32_t *>(packed), scales, w, nblocks, K / 32, K / kGroup);
+    return launch_status();
+}
+
+w3_status w3a16_gemm(const uint16_t *x, const int32_t *packed, const uint16_t *scales, uint16_t *y, int64_t M,
+                     int64_t N, int64_t K, w3_stream_t stream) {
+    if (!x || !packed || !scales || !y) return W3_ERR_NULL;
+    if (w3_status s = check_nk(N, K)) return s;
+    if (M < 1 || M > kMaxDim || M * K > kMaxElems || M * N > kMaxElems) return W3_ERR_SHAPE;
+    if (!aligned16(x) || !aligned16(packed) || !aligned16(scales) || !aligned16(y)) return W3_ERR_ALIGN;
+    const int64_t ybytes = M * N * 2;
+    if (overlaps(y, ybytes, x, M * K * 2) || overlaps(y, ybytes, packed, N * K * 3 / 8) ||
+        overlaps(y, ybytes, scales, N * (K / kGroup) * 2))
+        return W3_ERR_ALIAS;
+    int sms;
+    if (w3_status s = device_setup(&sms)) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    // Batches above 16 rows run as consecutive 16-row decode passes.
+    for (int64_t m0 = 0; m0 < M; m0 += 16) {
+        const int mb = static_cast<int>(std::min<int64_t>(16, M - m0));
+        if (w3_status s = launch_decode(x + m0 * K, packed, scales, y + m0 * N, mb, static_cast<int>(N),
+                                        static_cast<int>(K), sms, st))
+            return s;
+    }
+    return W3_OK;
+}
+
+w3_status w3_check_device_error(w3_stream_t stream) {
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return W3_ERR_CUDA;
+    unsigned int flag = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&flag, g_device_error, sizeof flag) != cudaSuccess) return W3_ERR_CUDA;
+    if (flag == 0) return W3_OK;
+    if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof zero) != cudaSuccess) return W3_ERR_CUDA;
+    return W3_ERR_TIMEOUT;
+}
+
+}  // extern "C"

@@ -1,0 +1,77 @@
+// format_kernels.cuh -- pack, unpack and fp32 dequantization of the exact-width
+// uint3 format (GSQ model card, section "Storage layout (why the HF UI shows
+// I32 + BF16)": [N,K] codes -> [N, 3K/32] int32, bf16 scales [N, K/128]).
+//
+// One thread handles one 32-code block = 3 consecutive words.  Rows hold K/32
+// whole blocks, so block b of the flattened matrix is words 3b..3b+2 and codes
+// 32b..32b+31 regardless of the row it falls in.  Bit order: code j of a block
+// is bits 3j..3j+2 of the block read as a little-endian 96-bit integer.
+#pragma once
+
+#include "common.cuh"
+
+namespace w3 {
+
+__device__ __forceinline__ unsigned __int128 load_block96(const uint32_t *__restrict__ p) {
+    return static_cast<unsigned __int128>(p[0]) | (static_cast<unsigned __int128>(p[1]) << 32) |
+           (static_cast<unsigned __int128>(p[2]) << 64);
+}
+
+__global__ void __launch_bounds__(256) pack_kernel(const uint8_t *__restrict__ codes, uint32_t *__restrict__ packed,
+                                                   int64_t nblocks) {
+    const int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (b >= nblocks) return;
+    const uint4 *src = reinterpret_cast<const uint4 *>(codes + 32 * b);
+    uint4 q[2] = {src[0], src[1]};
+    const uint8_t *c = reinterpret_cast<const uint8_t *>(q);
+    unsigned __int128 v = 0;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v |= static_cast<unsigned __int128>(c[j] & 7u) << (3 * j);
+    uint32_t *dst = packed + 3 * b;
+    dst[0] = static_cast<uint32_t>(v);
+    dst[1] = static_cast<uint32_t>(v >> 32);
+    dst[2] = static_cast<uint32_t>(v >> 64);
+}
+
+__global__ void __launch_bounds__(256) unpack_kernel(const uint32_t *__restrict__ packed,
+                                                     uint8_t *__restrict__ codes, int64_t nblocks) {
+    const int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (b >= nblocks) return;
+    const unsigned __int128 v = load_block96(packed + 3 * b);
+    uint4 q[2];
+    uint8_t *c = reinterpret_cast<uint8_t *>(q);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) c[j] = static_cast<uint8_t>((v >> (3 * j)) & 7u);
+    uint4 *dst = reinterpret_cast<uint4 *>(codes + 32 * b);
+    dst[0] = q[0];
+    dst[1] = q[1];
+}
+
+// w[n,k] = (c - 4) * s[n, k/128], exact in fp32.
+__global__ void __launch_bounds__(256) dequant_f32_kernel(const uint32_t *__restrict__ packed,
+                                                          const uint16_t *__restrict__ scales,
+                                                          float *__restrict__ w, int64_t nblocks,
+                                                          int64_t blocks_per_row, int64_t groups_per_row) {
+    const int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (b >= nblocks) return;
+    const int64_t n = b / blocks_per_row;
+    const int64_t t = b - n * blocks_per_row;  // block index within the row
+    const float s = bf16_bits_to_f32(scales[n * groups_per_row + t / 4]);
+    const unsigned __int128 v = load_block96(packed + 3 * b);
+    float4 *dst = reinterpret_cast<float4 *>(w + 32 * b);
+#pragma unroll
+    for (int j = 0; j < 32; j += 4) {
+        float4 o;
+        o.x = static_cast<float>(static_cast<int>((v >> (3 * j)) & 7u) - 4) * s;
+        o.y = static_cast<float>(static_cast<int>((v >> (3 * j + 3)) & 7u) - 4) * s;
+        o.z = static_cast<float>(static_cast<int>((v >> (3 * j + 6)) & 7u) - 4) * s;
+        o.w = static_cast<float>(static_cast<int>((v >> (3 * j + 9)) & 7u) - 4) * s;
+        dst[j / 4] = o;
+    }
+}
+
+inline unsigned grid_for(int64_t nblocks, int threads) {
+    return static_cast<unsigned>((nblocks + threads - 1) / threads);
+}
+
+}  // namespace w3
