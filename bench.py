@@ -41,11 +41,20 @@ BATCHES = (1, 4, 16)
 ROTATE = 5
 WORKLOAD = "Llama-3.1-70B gate_proj N=28672 K=8192, W3A16 g128 decode batch M=1,4,16"
 FALLBACK_HBM_GBS = 6650.0
-DECODE_SOURCES = ("w3a16_gemv_b200/csrc/decode_gemv.cuh", "w3a16_gemv_b200/csrc/common.cuh")
+DECODE_SOURCES = ("w3a16_gemv_b200/csrc/decode_gemv.cuh", "w3a16_gemv_b200/csrc/decode_streamk.cuh",
+                  "w3a16_gemv_b200/csrc/common.cuh")
 
 
 def algorithmic_bytes(M: int, N: int, K: int) -> int:
     return N * K * 3 // 8 + N * (K // 128) * 2 + M * K * 2 + M * N * 2
+
+
+def kernel_name(M: int) -> str:
+    """The kernel w3a16_gemm launches for a decode batch of M rows on the gate_proj shape."""
+    mt = 1 if M <= 1 else 2 if M <= 2 else 4 if M <= 4 else 8 if M <= 8 else 16
+    if mt <= 4:
+        return f"w3::decode_sk::decode_sk_kernel<{mt}> (M={M})"
+    return f"w3::decode::decode_kernel<{mt}> (M={M})"
 
 
 def step_bytes() -> int:
@@ -315,7 +324,7 @@ def run_gpu(args):
     traffic = recorded_traffic(dom["M"])
     roofline = {"bound": "hbm", "achieved": dom["GB/s"], "peak": peak, "unit": "GB/s",
                 "frac": dom["GB/s"] / peak, "traffic": traffic,
-                "kernel": f"w3::decode::decode_kernel<{1 if dom['M'] <= 8 else 2}> (M={dom['M']})",
+                "kernel": kernel_name(dom["M"]),
                 "algorithmic_bytes_per_launch": algorithmic_bytes(dom["M"], N_ROWS, K_COLS),
                 "peak_source": peak_src}
 

@@ -13,10 +13,14 @@
 #include "../../include/w3a16.h"
 #include "common.cuh"
 #include "decode_gemv.cuh"
+#include "decode_streamk.cuh"
 #include "format_kernels.cuh"
 
 #ifndef W3_DECODE_TMA2D
 #define W3_DECODE_TMA2D 1
+#endif
+#ifndef W3_DECODE_STREAMK
+#define W3_DECODE_STREAMK 1
 #endif
 
 namespace w3 {
@@ -61,6 +65,17 @@ w3_status device_setup(int *num_sms) {
             reinterpret_cast<const void *>(decode::decode_kernel<8>),
             reinterpret_cast<const void *>(decode::decode_kernel<16>),
         };
+        const void *sk_kernels[] = {
+            reinterpret_cast<const void *>(decode_sk::decode_sk_kernel<1>),
+            reinterpret_cast<const void *>(decode_sk::decode_sk_kernel<2>),
+            reinterpret_cast<const void *>(decode_sk::decode_sk_kernel<4>),
+        };
+        for (const void *k : sk_kernels) {
+            if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, optin) != cudaSuccess) {
+                st.status = W3_ERR_CUDA;
+                return;
+            }
+        }
         for (const void *k : kernels) {
             if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, optin) != cudaSuccess) {
                 st.status = W3_ERR_CUDA;
@@ -102,6 +117,56 @@ w3_status check_nk(int64_t N, int64_t K) {
 
 w3_status launch_status() {
     return cudaGetLastError() == cudaSuccess ? W3_OK : W3_ERR_CUDA;
+}
+
+// A [rows][box_words] box over the packed matrix [N][3K/32] u32.
+w3_status encode_packed_map(CUtensorMap *map, const int32_t *packed, int64_t N, int64_t words, uint32_t box_words,
+                            uint32_t box_rows) {
+    PFN_cuTensorMapEncodeTiled enc = tensor_map_encoder();
+    if (!enc) return W3_ERR_CUDA;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(words), static_cast<cuuint64_t>(N)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(words * 4)};
+    cuuint32_t box[2] = {box_words, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<int32_t *>(packed), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS
+               ? W3_OK
+               : W3_ERR_CUDA;
+}
+
+w3_status launch_decode_sk(const uint16_t *x, const int32_t *packed, const uint16_t *scales, uint16_t *y, int M,
+                           int N, int K, int num_sms, cudaStream_t stream) {
+    const decode_sk::LaunchPlan P = decode_sk::plan(M, N, K, num_sms);
+    decode_sk::Params prm;
+    const int64_t words = static_cast<int64_t>(K) * 3 / 32;
+    if (w3_status s = encode_packed_map(&prm.tmap1, packed, N, words, decode_sk::kPitch1, decode_sk::kBlockRows))
+        return s;
+    prm.tmap3 = prm.tmap1;  // only used when a segment has 3 groups left, which needs K >= 384
+    if (words >= decode_sk::kPitch3) {
+        if (w3_status s = encode_packed_map(&prm.tmap3, packed, N, words, decode_sk::kPitch3, decode_sk::kBlockRows))
+            return s;
+    }
+    prm.x = x;
+    prm.scales = scales;
+    prm.y = y;
+    prm.M = M;
+    prm.N = N;
+    prm.K = K;
+    prm.ctas = P.ctas;
+    prm.depth = P.depth;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(P.ctas, 1, 1);
+    cfg.blockDim = dim3(decode_sk::kWarps * 32, 1, 1);
+    cfg.dynamicSmemBytes = P.smem_bytes;
+    cfg.stream = stream;
+    cudaError_t e;
+    switch (P.mt) {
+        case 1: e = cudaLaunchKernelEx(&cfg, decode_sk::decode_sk_kernel<1>, prm); break;
+        case 2: e = cudaLaunchKernelEx(&cfg, decode_sk::decode_sk_kernel<2>, prm); break;
+        default: e = cudaLaunchKernelEx(&cfg, decode_sk::decode_sk_kernel<4>, prm); break;
+    }
+    return e == cudaSuccess ? W3_OK : W3_ERR_CUDA;
 }
 
 w3_status launch_decode(const uint16_t *x, const int32_t *packed, const uint16_t *scales, uint16_t *y, int M,
@@ -245,9 +310,12 @@ w3_status w3a16_gemm(const uint16_t *x, const int32_t *packed, const uint16_t *s
     // Batches above 16 rows run as consecutive 16-row decode passes.
     for (int64_t m0 = 0; m0 < M; m0 += 16) {
         const int mb = static_cast<int>(std::min<int64_t>(16, M - m0));
-        if (w3_status s = launch_decode(x + m0 * K, packed, scales, y + m0 * N, mb, static_cast<int>(N),
-                                        static_cast<int>(K), sms, st))
-            return s;
+        const bool sk = W3_DECODE_STREAMK && decode_sk::applicable(mb, static_cast<int>(N), static_cast<int>(K));
+        w3_status s = sk ? launch_decode_sk(x + m0 * K, packed, scales, y + m0 * N, mb, static_cast<int>(N),
+                                            static_cast<int>(K), sms, st)
+                         : launch_decode(x + m0 * K, packed, scales, y + m0 * N, mb, static_cast<int>(N),
+                                         static_cast<int>(K), sms, st);
+        if (s) return s;
     }
     return W3_OK;
 }

@@ -144,10 +144,13 @@ __device__ __forceinline__ float4 ld_dsmem_f4(uint32_t addr) {
 
 // ---- bit manipulation ----------------------------------------------------------------
 
-// (a & b) | c in one LOP3.
-__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t b, uint32_t c) {
+// (a & MASK) | c in exactly one LOP3: the mask is the instruction's immediate
+// and c stays in a register.  (Written as C, the two constants would not both
+// fit a single LOP3 and the compiler splits it in two.)
+template <uint32_t MASK>
+__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t c) {
     uint32_t d;
-    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "n"(MASK), "r"(c));
     return d;
 }
 

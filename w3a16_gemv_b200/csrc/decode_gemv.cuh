@@ -59,6 +59,7 @@ constexpr int kDepth = W3_DECODE_DEPTH;             // ring stages per warp
 static_assert(kStageGroups % 2 == 1, "an odd number of groups per stage keeps the row pitch conflict-free");
 constexpr int kRowPitchWords = kStageGroups * kWordsPerGroup;   // 36 for 3 groups
 constexpr int kStageBytes = kRowsPerWarp * kRowPitchWords * 4;  // 4608 for 3 groups
+static_assert(kStageBytes % 128 == 0, "a tiled TMA destination in shared memory must be 128-byte aligned");
 constexpr int kXsBudgetBytes = 64 * 1024;                       // prepared-x budget per CTA
 constexpr int kMaxCluster = 8;
 
@@ -94,10 +95,12 @@ __host__ __device__ constexpr int code_shift(int j) {
 
 constexpr uint32_t kMagic = 0x43004300u;  // bf16x2 (128.0, 128.0)
 
+
 // Unpack one 96-bit block (w0, w1, w2) into the 16 bf16x2 pair registers.
 // Window s (a shift of the block by s bits) feeds the pairs whose codes sit at
 // window bits e_lo and 16 + e_hi.
 __device__ __forceinline__ void unpack_block(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t (&a)[16]) {
+    const uint32_t magic = kMagic;
     const uint32_t wm4 = w0 << 4;                     // s = -4
     const uint32_t w_2 = w0 >> 2;                     // s = 2
     const uint32_t w_8 = w0 >> 8;                     // s = 8
@@ -107,22 +110,46 @@ __device__ __forceinline__ void unpack_block(uint32_t w0, uint32_t w1, uint32_t 
     const uint32_t w44 = __funnelshift_r(w1, w2, 12); // s = 44
     const uint32_t w68 = w2 >> 4;                     // s = 68
     const uint32_t w74 = w2 >> 10;                    // s = 74
-    a[0] = and_or(wm4, pair_mask(4, 0), kMagic);
-    a[1] = and_or(w_2, pair_mask(1, 3), kMagic);
-    a[2] = and_or(w_2, pair_mask(4, 0), kMagic);
-    a[3] = and_or(w_8, pair_mask(1, 3), kMagic);
-    a[4] = and_or(w11, pair_mask(4, 3), kMagic);
-    a[5] = and_or(w20, pair_mask(4, 0), kMagic);
-    a[6] = and_or(w1, pair_mask(1, 3), kMagic);
-    a[7] = and_or(w38, pair_mask(1, 0), kMagic);
-    a[8] = and_or(w38, pair_mask(4, 3), kMagic);
-    a[9] = and_or(w44, pair_mask(1, 3), kMagic);
-    a[10] = and_or(w44, pair_mask(4, 0), kMagic);
-    a[11] = and_or(w2, pair_mask(2, 1), kMagic);
-    a[12] = and_or(w68, pair_mask(1, 0), kMagic);
-    a[13] = and_or(w68, pair_mask(4, 3), kMagic);
-    a[14] = and_or(w74, pair_mask(1, 3), kMagic);
-    a[15] = and_or(w74, pair_mask(4, 0), kMagic);
+    a[0] = and_or<pair_mask(4, 0)>(wm4, magic);
+    a[1] = and_or<pair_mask(1, 3)>(w_2, magic);
+    a[2] = and_or<pair_mask(4, 0)>(w_2, magic);
+    a[3] = and_or<pair_mask(1, 3)>(w_8, magic);
+    a[4] = and_or<pair_mask(4, 3)>(w11, magic);
+    a[5] = and_or<pair_mask(4, 0)>(w20, magic);
+    a[6] = and_or<pair_mask(1, 3)>(w1, magic);
+    a[7] = and_or<pair_mask(1, 0)>(w38, magic);
+    a[8] = and_or<pair_mask(4, 3)>(w38, magic);
+    a[9] = and_or<pair_mask(1, 3)>(w44, magic);
+    a[10] = and_or<pair_mask(4, 0)>(w44, magic);
+    a[11] = and_or<pair_mask(2, 1)>(w2, magic);
+    a[12] = and_or<pair_mask(1, 0)>(w68, magic);
+    a[13] = and_or<pair_mask(4, 3)>(w68, magic);
+    a[14] = and_or<pair_mask(1, 3)>(w74, magic);
+    a[15] = and_or<pair_mask(4, 0)>(w74, magic);
+}
+
+// Pair I of a block (the I-th register of unpack_block), computed on its own so
+// that callers can interleave the unpack with the MMAs; with the index known at
+// compile time the windows shared by two pairs are computed once.
+template <int I>
+__device__ __forceinline__ uint32_t unpack_pair(uint32_t w0, uint32_t w1, uint32_t w2) {
+    const uint32_t magic = kMagic;
+    if constexpr (I == 0) return and_or<pair_mask(4, 0)>(w0 << 4, magic);
+    if constexpr (I == 1) return and_or<pair_mask(1, 3)>(w0 >> 2, magic);
+    if constexpr (I == 2) return and_or<pair_mask(4, 0)>(w0 >> 2, magic);
+    if constexpr (I == 3) return and_or<pair_mask(1, 3)>(w0 >> 8, magic);
+    if constexpr (I == 4) return and_or<pair_mask(4, 3)>(__funnelshift_r(w0, w1, 11), magic);
+    if constexpr (I == 5) return and_or<pair_mask(4, 0)>(__funnelshift_r(w0, w1, 20), magic);
+    if constexpr (I == 6) return and_or<pair_mask(1, 3)>(w1, magic);
+    if constexpr (I == 7) return and_or<pair_mask(1, 0)>(w1 >> 6, magic);
+    if constexpr (I == 8) return and_or<pair_mask(4, 3)>(w1 >> 6, magic);
+    if constexpr (I == 9) return and_or<pair_mask(1, 3)>(__funnelshift_r(w1, w2, 12), magic);
+    if constexpr (I == 10) return and_or<pair_mask(4, 0)>(__funnelshift_r(w1, w2, 12), magic);
+    if constexpr (I == 11) return and_or<pair_mask(2, 1)>(w2, magic);
+    if constexpr (I == 12) return and_or<pair_mask(1, 0)>(w2 >> 4, magic);
+    if constexpr (I == 13) return and_or<pair_mask(4, 3)>(w2 >> 4, magic);
+    if constexpr (I == 14) return and_or<pair_mask(1, 3)>(w2 >> 10, magic);
+    return and_or<pair_mask(4, 0)>(w2 >> 10, magic);
 }
 
 // x * 2^-e as bf16 bits (exact: only the exponent changes).
@@ -310,7 +337,8 @@ __global__ void __launch_bounds__(kWarps * 32, W3_DECODE_MIN_CTAS) decode_kernel
             const int ng = min(kStageGroups, ng_chunk - gs);
             const uint32_t parity = (phase_bits >> slot) & 1u;
             phase_bits ^= 1u << slot;
-            if (!mbar_wait_bounded(bar0 + 8 * slot, parity)) ok = false;
+            // warp-uniform: a timeout seen by any lane stops the whole warp
+            ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar0 + 8 * slot, parity) && ok);
             if (!ok) continue;  // drain the copies still in flight, compute nothing
             const uint32_t *st = reinterpret_cast<const uint32_t *>(ring + slot * kStageBytes);
 #pragma unroll
