@@ -44,6 +44,9 @@ SMALL = [
     (1, 64, 28672, "gsq_5level", "absnormal", "normal_outliers"),
     (17, 50, 512, "uniform8", "lognormal", "normal"),
     (40, 96, 1280, "uniform8", "lognormal", "normal"),
+    (256, 256, 256, "uniform8", "lognormal", "normal"),
+    (300, 1000, 1024, "gsq_5level", "absnormal", "normal_outliers"),
+    (513, 200, 384, "uniform8", "lognormal", "normal"),
 ]
 
 

@@ -15,12 +15,16 @@
 #include "decode_gemv.cuh"
 #include "decode_streamk.cuh"
 #include "format_kernels.cuh"
+#include "prefill_gemm.cuh"
 
 #ifndef W3_DECODE_TMA2D
 #define W3_DECODE_TMA2D 1
 #endif
 #ifndef W3_DECODE_STREAMK
 #define W3_DECODE_STREAMK 1
+#endif
+#ifndef W3_PREFILL_TCGEN05
+#define W3_PREFILL_TCGEN05 1
 #endif
 
 namespace w3 {
@@ -75,6 +79,11 @@ w3_status device_setup(int *num_sms) {
                 st.status = W3_ERR_CUDA;
                 return;
             }
+        }
+        if (cudaFuncSetAttribute(prefill::prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 prefill::SmemLayout::total) != cudaSuccess) {
+            st.status = W3_ERR_CUDA;
+            return;
         }
         for (const void *k : kernels) {
             if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, optin) != cudaSuccess) {
@@ -167,6 +176,36 @@ w3_status launch_decode_sk(const uint16_t *x, const int32_t *packed, const uint1
         default: e = cudaLaunchKernelEx(&cfg, decode_sk::decode_sk_kernel<4>, prm); break;
     }
     return e == cudaSuccess ? W3_OK : W3_ERR_CUDA;
+}
+
+w3_status launch_prefill(const uint16_t *x, const int32_t *packed, const uint16_t *scales, uint16_t *y, int M,
+                         int N, int K, int num_sms, cudaStream_t stream) {
+    const prefill::LaunchPlan P = prefill::plan(M, N, num_sms);
+    prefill::Params prm;
+    PFN_cuTensorMapEncodeTiled enc = tensor_map_encoder();
+    if (!enc) return W3_ERR_CUDA;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+    cuuint32_t box[2] = {prefill::kStageK, prefill::kUmmaM};
+    cuuint32_t estr[2] = {1, 1};
+    if (enc(&prm.tmap_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t *>(x), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return W3_ERR_CUDA;
+    prm.packed = reinterpret_cast<const uint32_t *>(packed);
+    prm.scales = scales;
+    prm.y = y;
+    prm.M = M;
+    prm.N = N;
+    prm.K = K;
+    prm.tile_n = P.tile_n;
+    prm.idesc = prefill::make_idesc(prefill::kUmmaM, P.tile_n);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = P.grid;
+    cfg.blockDim = dim3(prefill::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = prefill::SmemLayout::total;
+    cfg.stream = stream;
+    return cudaLaunchKernelEx(&cfg, prefill::prefill_kernel, prm) == cudaSuccess ? W3_OK : W3_ERR_CUDA;
 }
 
 w3_status launch_decode(const uint16_t *x, const int32_t *packed, const uint16_t *scales, uint16_t *y, int M,
@@ -307,7 +346,10 @@ w3_status w3a16_gemm(const uint16_t *x, const int32_t *packed, const uint16_t *s
     int sms;
     if (w3_status s = device_setup(&sms)) return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    // Batches above 16 rows run as consecutive 16-row decode passes.
+    if (M > 16 && W3_PREFILL_TCGEN05)
+        return launch_prefill(x, packed, scales, y, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), sms,
+                              st);
+    // Batches above 16 rows without the tensor-core path run as 16-row decode passes.
     for (int64_t m0 = 0; m0 < M; m0 += 16) {
         const int mb = static_cast<int>(std::min<int64_t>(16, M - m0));
         const bool sk = W3_DECODE_STREAMK && decode_sk::applicable(mb, static_cast<int>(N), static_cast<int>(K));

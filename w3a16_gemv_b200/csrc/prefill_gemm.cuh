@@ -1,0 +1,355 @@
+// prefill_gemm.cuh -- y = x * W^T for batches M > 16 on the 5th-generation
+// tensor cores (tcgen05), W in the exact-width uint3 / group-128 / bf16-scale
+// format of the GSQ model card ("Storage layout" section).
+//
+// A prefill batch makes the product a real dense contraction (2*M*N*K flops
+// over (3/8)*N*K bytes of weights), so it runs as a GEMM whose B operand is
+// produced on the fly:
+//
+//  * CTA tile: 256 rows of x (two 128-row UMMA tiles) x BN rows of W (BN a
+//    multiple of 32, at most 256, chosen per shape to fill the last wave),
+//    over K in stages of 64.  The fp32 accumulators live in tensor memory:
+//    2 x BN columns of the 512 the CTA allocates.
+//  * A (x): one tiled TMA copy per 128-row tile and stage, 128-byte swizzle,
+//    the canonical K-major layout the UMMA descriptors describe.
+//  * B (W): 8 dequantizing warps, one W row per thread.  A stage of a row is
+//    64 codes = 6 packed words (loaded one stage ahead).  Codes are expanded
+//    in natural k order four at a time: the 12 bits of two code pairs times
+//    0x2001 place each pair's second code 13 bits above its first, so one
+//    LOP3 (mask | bf16 128.0) per pair gives (128 + c_k, 128 + c_k+1) exactly;
+//    a bf16x2 subtract of 132 gives the levels q = c - 4, and a bf16x2
+//    multiply by the group scale gives bf16(q * s), rounded once.  The row is
+//    stored into the stage's B buffer in the same 128-byte-swizzled K-major
+//    layout, then made visible to the tensor cores' async proxy.
+//  * One thread issues tcgen05.mma (kind::f16, bf16 x bf16 -> fp32) for both
+//    128-row tiles and commits each stage back to the producers.
+//  * Epilogue: the 8 warps read the accumulators with tcgen05.ld, round to
+//    bf16 and store y.
+// All waits are bounded; a timeout is recorded and the CTA winds down.
+#pragma once
+
+#include "common.cuh"
+
+namespace w3 {
+namespace prefill {
+
+constexpr int kTileM = 256;          // rows of x per CTA (two UMMA M=128 tiles)
+constexpr int kUmmaM = 128;
+constexpr int kMaxTileN = 256;       // rows of W per CTA at most
+constexpr int kStageK = 64;          // k per pipeline stage = one 128-byte swizzle atom of bf16
+constexpr int kStages = 3;
+constexpr int kDequantWarps = 8;     // one W row per thread: BN <= 256
+constexpr int kThreads = (2 + kDequantWarps) * 32;
+constexpr int kTmemCols = 512;
+constexpr int kABytes = kUmmaM * kStageK * 2;     // 16 KB per 128-row tile and stage
+constexpr int kBBytes = kMaxTileN * kStageK * 2;  // 32 KB per stage (BN rows used)
+constexpr int kStageWords = kStageK * 3 / 32;     // 6 packed words per row and stage
+
+struct SmemLayout {
+    // all operand buffers are 1024-byte aligned (the 128-byte swizzle period)
+    static constexpr int a_off = 0;                                  // [kStages][2][kABytes]
+    static constexpr int b_off = a_off + kStages * 2 * kABytes;      // [kStages][kBBytes]
+    static constexpr int bar_off = b_off + kStages * kBBytes;        // u64 full_a, full_b, empty [kStages], acc
+    static constexpr int tmem_slot_off = bar_off + (3 * kStages + 1) * 8;
+    static constexpr int total = tmem_slot_off + 16 + 1024;          // + slack to align the base to 1024
+};
+
+struct Params {
+    CUtensorMap tmap_x;  // x [M][K] bf16, box [128 rows][64 k], 128-byte swizzle
+    const uint32_t *packed;
+    const uint16_t *scales;
+    uint16_t *y;
+    int M, N, K;
+    int tile_n;      // BN, a multiple of 32
+    uint32_t idesc;  // UMMA instruction descriptor for M=128, N=BN
+};
+
+// K-major operand tile with 128-byte rows, 128-byte swizzle, 8-row groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);  // start address (16-byte units)
+    d |= static_cast<uint64_t>(1) << 16;                  // leading byte offset (unused for swizzled K-major)
+    d |= static_cast<uint64_t>(1024 >> 4) << 32;          // stride byte offset: next 8-row group
+    d |= static_cast<uint64_t>(1) << 46;                  // descriptor version (Blackwell)
+    d |= static_cast<uint64_t>(2) << 61;                  // layout: 128-byte swizzle
+    return d;
+}
+
+// bf16 x bf16 -> fp32, both operands K-major, D in tensor memory.
+__host__ __device__ constexpr uint32_t make_idesc(int m, int n) {
+    return (1u << 4)       // D format: f32
+           | (1u << 7)     // A format: bf16
+           | (1u << 10)    // B format: bf16
+           | (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(m >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// 32 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+          "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+          "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Bits [12q, 12q+12) of the 192-bit stage stream w[0..5]: codes 4q..4q+3.
+template <int Q>
+__device__ __forceinline__ uint32_t quad_bits(const uint32_t (&w)[kStageWords]) {
+    constexpr int b = 12 * Q, i = b / 32, s = b % 32;
+    if constexpr (s + 12 <= 32) return (w[i] >> s) & 0xFFFu;
+    else return __funnelshift_r(w[i], w[i + 1], s) & 0xFFFu;
+}
+
+__device__ __forceinline__ uint32_t bf16x2_sub_mul(uint32_t v, uint32_t sub, uint32_t mul) {
+    uint32_t q, r;
+    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(q) : "r"(v), "r"(sub));  // exact: c - 4
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(q), "r"(mul));  // bf16(q * s), one rounding
+    return r;
+}
+
+// Expand one row's stage (64 codes) into 32 bf16x2 words of bf16(q*s), natural k order.
+template <int Q>
+__device__ __forceinline__ void expand_quads(const uint32_t (&w)[kStageWords], uint32_t s2, uint32_t (&out)[32]) {
+    if constexpr (Q < 16) {
+        constexpr uint32_t kMagic2 = 0x43004300u;  // bf16x2 (128, 128)
+        constexpr uint32_t kSub = 0x43044304u;     // bf16x2 (132, 132)
+        const uint32_t x = quad_bits<Q>(w) * 0x2001u;  // second code of each pair 13 bits above the first
+        out[2 * Q] = bf16x2_sub_mul(and_or<0x00070007u>(x, kMagic2), kSub, s2);
+        out[2 * Q + 1] = bf16x2_sub_mul(and_or<0x00070007u>(x >> 6, kMagic2), kSub, s2);
+        expand_quads<Q + 1>(w, s2, out);
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_constant__ Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_addr(smem);
+    const uint32_t a_base = sbase + SmemLayout::a_off;
+    const uint32_t b_base = sbase + SmemLayout::b_off;
+    const uint32_t bar_full_a = sbase + SmemLayout::bar_off;
+    const uint32_t bar_full_b = bar_full_a + 8 * kStages;
+    const uint32_t bar_empty = bar_full_b + 8 * kStages;
+    const uint32_t bar_acc = bar_empty + 8 * kStages;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + SmemLayout::tmem_slot_off);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int m0 = blockIdx.y * kTileM;
+    const int n0 = blockIdx.x * p.tile_n;
+    const int nstages = p.K / kStageK;
+    const int G = p.K / kGroup;
+    const int W = G * kWordsPerGroup;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(bar_full_a + 8 * s, 1);
+            mbar_init(bar_full_b + 8 * s, kDequantWarps * 32);
+            mbar_init(bar_empty + 8 * s, 1);
+        }
+        mbar_init(bar_acc, 1);
+        mbar_init_fence();
+    }
+    if (warp == 1) {  // allocate the accumulators
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_addr(tmem_slot)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    bool ok = true;
+
+    if (warp == 0) {
+        // ---- A producer: x tiles by TMA ----
+        if (lane == 0) {
+            for (int s = 0; s < nstages && ok; ++s) {
+                const int slot = s % kStages;
+                const uint32_t round = static_cast<uint32_t>(s / kStages);
+                ok = mbar_wait_bounded(bar_empty + 8 * slot, (round & 1u) ^ 1u);
+                if (!ok) break;
+                mbar_arrive_expect_tx(bar_full_a + 8 * slot, 2 * kABytes);
+                const uint32_t dst = a_base + slot * 2 * kABytes;
+                tma_load_2d(dst, &p.tmap_x, s * kStageK, m0, bar_full_a + 8 * slot);
+                tma_load_2d(dst + kABytes, &p.tmap_x, s * kStageK, m0 + kUmmaM, bar_full_a + 8 * slot);
+            }
+        }
+    } else if (warp == 1) {
+        // ---- MMA issuer ----
+        if (lane == 0) {
+            for (int s = 0; s < nstages && ok; ++s) {
+                const int slot = s % kStages;
+                const uint32_t par = static_cast<uint32_t>(s / kStages) & 1u;
+                ok = mbar_wait_bounded(bar_full_a + 8 * slot, par) && mbar_wait_bounded(bar_full_b + 8 * slot, par);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t a0 = a_base + slot * 2 * kABytes;
+                const uint32_t b0 = b_base + slot * kBBytes;
+#pragma unroll
+                for (int kk = 0; kk < kStageK / 16; ++kk) {
+                    const uint64_t bd = sw128_kmajor_desc(b0 + kk * 32);
+                    const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
+                    umma_bf16(tmem, sw128_kmajor_desc(a0 + kk * 32), bd, p.idesc, acc);
+                    umma_bf16(tmem + static_cast<uint32_t>(p.tile_n), sw128_kmajor_desc(a0 + kABytes + kk * 32), bd,
+                              p.idesc, acc);
+                }
+                umma_commit(bar_empty + 8 * slot);  // frees the stage once these MMAs have read it
+            }
+            umma_commit(bar_acc);  // all accumulation done
+        }
+    } else {
+        // ---- B producers: dequantize one W row per thread ----
+        const int t = threadIdx.x - 64;  // 0..255
+        const int n = n0 + t;
+        const bool row_ok = (t < p.tile_n) && (n < p.N);
+        const uint32_t *prow = p.packed + static_cast<int64_t>(row_ok ? n : 0) * W;
+        const uint16_t *srow = p.scales + static_cast<int64_t>(row_ok ? n : 0) * G;
+        uint32_t w[kStageWords] = {};
+        uint32_t s_next = 0;
+        auto load = [&](int s, uint32_t (&dst)[kStageWords], uint32_t &sc) {
+            if (row_ok && s < nstages) {
+                const uint2 *src = reinterpret_cast<const uint2 *>(prow + s * kStageWords);
+#pragma unroll
+                for (int i = 0; i < 3; ++i) {
+                    const uint2 v = __ldg(src + i);
+                    dst[2 * i] = v.x;
+                    dst[2 * i + 1] = v.y;
+                }
+                const uint32_t h = __ldg(srow + s / 2);  // one scale per 128 = two stages
+                sc = h | (h << 16);
+            }
+        };
+        load(0, w, s_next);
+        for (int s = 0; s < nstages && ok; ++s) {
+            uint32_t cur[kStageWords];
+#pragma unroll
+            for (int i = 0; i < kStageWords; ++i) cur[i] = w[i];
+            const uint32_t s2 = s_next;
+            load(s + 1, w, s_next);  // prefetch the next stage
+            uint32_t out[32];
+            if (row_ok) {
+                expand_quads<0>(cur, s2, out);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) out[i] = 0u;
+            }
+            const int slot = s % kStages;
+            const uint32_t round = static_cast<uint32_t>(s / kStages);
+            ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar_empty + 8 * slot, (round & 1u) ^ 1u));
+            if (!ok) break;
+            if (t < p.tile_n) {
+                const uint32_t row = b_base + slot * kBBytes + t * 128;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const uint32_t dst = row + ((j ^ (t & 7)) << 4);
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(out[4 * j]),
+                                 "r"(out[4 * j + 1]), "r"(out[4 * j + 2]), "r"(out[4 * j + 3])
+                                 : "memory");
+                }
+            }
+            fence_async_smem();
+            mbar_arrive(bar_full_b + 8 * slot);
+        }
+
+        // ---- epilogue: TMEM -> bf16 -> y ----
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar_acc, 0));
+        tc_fence_after();
+        if (ok) {
+            const int quarter = warp & 3;           // TMEM lanes 32*quarter .. +31
+            const int sub = (warp - 2) / 4;         // warps 2-5: tile 0, warps 6-9: tile 1
+            const int m = m0 + sub * kUmmaM + quarter * 32 + lane;
+            const uint32_t tbase = tmem + (static_cast<uint32_t>(quarter * 32) << 16) +
+                                   static_cast<uint32_t>(sub * p.tile_n);
+            for (int c0 = 0; c0 < p.tile_n; c0 += 32) {
+                uint32_t v[32];
+                tmem_ld32(tbase + c0, v);
+                if (m < p.M) {
+                    uint16_t *yrow = p.y + static_cast<int64_t>(m) * p.N;
+                    const int nb = n0 + c0;
+                    if (nb + 32 <= p.N && (p.N % 8) == 0) {
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            pk[i] = static_cast<uint32_t>(f32_to_bf16_rn(__uint_as_float(v[2 * i]))) |
+                                    (static_cast<uint32_t>(f32_to_bf16_rn(__uint_as_float(v[2 * i + 1]))) << 16);
+                        uint4 *dst = reinterpret_cast<uint4 *>(yrow + nb);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                    } else {
+                        for (int i = 0; i < 32; ++i)
+                            if (nb + i < p.N) yrow[nb + i] = f32_to_bf16_rn(__uint_as_float(v[i]));
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+    }
+}
+
+struct LaunchPlan {
+    int tile_n;
+    dim3 grid;
+};
+
+// BN: a multiple of 32 in [128, 256] that leaves the last wave fullest (a
+// multiple of 32 so that the epilogue's 32-column TMEM reads never cross into
+// the next tile's columns).
+inline LaunchPlan plan(int M, int N, int num_sms) {
+    LaunchPlan P;
+    const int mt = (M + kTileM - 1) / kTileM;
+    int best = kMaxTileN;
+    double best_eff = -1.0;
+    for (int bn = kMaxTileN; bn >= 128; bn -= 32) {
+        const int tiles = mt * ((N + bn - 1) / bn);
+        const int waves = (tiles + num_sms - 1) / num_sms;
+        // useful work over scheduled work, counting padding of the last N tile
+        const double eff = static_cast<double>(M) * N / (static_cast<double>(waves) * num_sms * kTileM * bn);
+        if (eff > best_eff + 1e-9) {
+            best_eff = eff;
+            best = bn;
+        }
+    }
+    if (N < 128) best = (N + 31) / 32 * 32;
+    P.tile_n = best;
+    P.grid = dim3((N + best - 1) / best, mt, 1);
+    return P;
+}
+
+}  // namespace prefill
+}  // namespace w3
