@@ -226,6 +226,92 @@ def run_reference(args):
 # GPU arm
 # --------------------------------------------------------------------------------------
 
+def measured_tensor_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), "measured (MEASURED_PEAKS.json bf16_tflops: cuBLAS bf16 GEMM, burst)"
+    except (OSError, KeyError, ValueError):
+        return 1590.0, "fallback (1.59 PFLOP/s earlier measurement on this pool)"
+
+
+def run_prefill(args):
+    """Prefill workload: y = x W^T at M=2048, N=28672, K=8192 (one call per step)."""
+    import torch
+
+    from w3a16_gemv_b200 import build as wbuild
+    from w3a16_gemv_b200 import w3_check_device_error, w3_pack, w3a16_gemm
+    from w3a16_gemv_b200.inputs import make_problem
+
+    world, rank, local = dist_setup()
+    if world > 1:
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if not os.path.exists(wbuild.LIB):
+        wbuild.build()
+    M, N, K = 2048, N_ROWS, K_COLS
+    p = make_problem(M, N, K, "uniform8", "lognormal", "normal", seed=0)
+    packed = w3_pack(torch.from_numpy(p.codes).to(dev))
+    scales = torch.from_numpy(p.scales_bf16.view(np.int16)).view(torch.bfloat16).to(dev)
+    x = torch.from_numpy(p.x_bf16.view(np.int16)).view(torch.bfloat16).to(dev)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        w3a16_gemm(x, packed, scales, out=y)
+    torch.cuda.synchronize()
+    w3_check_device_error()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.02)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    w0 = time.perf_counter()
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        w3a16_gemm(x, packed, scales, out=y)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    w1 = time.perf_counter()
+    sampler.stop()
+    w3_check_device_error()
+    per_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = ev[0][0].elapsed_time(ev[-1][1])
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    flop = 2.0 * M * N * K
+    value = flop * args.steps * world / (total_ms * 1e-3) / 1e12
+    peak, src = measured_tensor_peak()
+    achieved = flop / (statistics.mean(per_ms) * 1e-3) / 1e12
+    line = {
+        "metric": "W3A16 g128 prefill GEMM TFLOP/s (M=2048, Llama-70B gate_proj)", "value": value,
+        "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "prefill M=2048 N=28672 K=8192 (Llama-3.1-70B gate_proj)", "M": M, "N": N, "K": K,
+                   "l2": "inputs larger than L2 (x 33.6 MB + weights 91.8 MB + y 117.4 MB)"},
+        "us_per_call": 1e3 * statistics.median(per_ms),
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": None, "kernel": "w3::prefill::prefill_kernel",
+                     "peak_source": src, "frac_of_nominal_2250": achieved / 2250.0},
+        "gpu_launches": args.steps,
+        "clocks": sampler.summary(w0, w1),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
 def run_gpu(args):
     import torch
 
@@ -399,11 +485,15 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of CPU oracle work for cpu_baseline")
     ap.add_argument("--ref-budget", type=float, default=3.0, help="seconds of oracle work per reference step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", choices=("gate_decode", "prefill"), default="gate_decode",
+                    help="gate_decode: the headline decode step (default); prefill: M=2048 tensor-core GEMM")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload == "prefill":
+        return run_prefill(args)
     return run_gpu(args)
 
 
