@@ -14,6 +14,7 @@
 #include "common.cuh"
 #include "decode_gemv.cuh"
 #include "decode_streamk.cuh"
+#include "decode_tcgen05.cuh"
 #include "format_kernels.cuh"
 #include "prefill_gemm.cuh"
 
@@ -25,6 +26,10 @@
 #endif
 #ifndef W3_PREFILL_TCGEN05
 #define W3_PREFILL_TCGEN05 1
+#endif
+// Smallest decode batch that uses the tcgen05 decode kernel (above 16: never).
+#ifndef W3_DECODE_TC_MIN_M
+#define W3_DECODE_TC_MIN_M 5
 #endif
 
 namespace w3 {
@@ -79,6 +84,11 @@ w3_status device_setup(int *num_sms) {
                 st.status = W3_ERR_CUDA;
                 return;
             }
+        }
+        if (cudaFuncSetAttribute(decode_tc::decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 decode_tc::SmemLayout::total) != cudaSuccess) {
+            st.status = W3_ERR_CUDA;
+            return;
         }
         if (cudaFuncSetAttribute(prefill::prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  prefill::SmemLayout::total) != cudaSuccess) {
@@ -176,6 +186,40 @@ w3_status launch_decode_sk(const uint16_t *x, const int32_t *packed, const uint1
         default: e = cudaLaunchKernelEx(&cfg, decode_sk::decode_sk_kernel<4>, prm); break;
     }
     return e == cudaSuccess ? W3_OK : W3_ERR_CUDA;
+}
+
+// Tensor-core decode (tcgen05, weights as the MMA's M dimension).  Returns
+// W3_ERR_UNSUPPORTED, without launching, when a tensor map for this shape
+// cannot be encoded; the caller then uses the mma.sync kernels.
+w3_status launch_decode_tc(const uint16_t *x, const int32_t *packed, const uint16_t *scales, uint16_t *y, int M,
+                           int N, int K, cudaStream_t stream) {
+    decode_tc::Params prm;
+    const int64_t words = static_cast<int64_t>(K) * 3 / 32;
+    if (N < decode_tc::kRows || words < decode_tc::kPitch) return W3_ERR_UNSUPPORTED;
+    if (encode_packed_map(&prm.tmap_w, packed, N, words, decode_tc::kPitch, decode_tc::kRows) != W3_OK)
+        return W3_ERR_UNSUPPORTED;
+    PFN_cuTensorMapEncodeTiled enc = tensor_map_encoder();
+    if (!enc) return W3_ERR_CUDA;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+    cuuint32_t box[2] = {64, decode_tc::kBatch};
+    cuuint32_t estr[2] = {1, 1};
+    if (enc(&prm.tmap_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t *>(x), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return W3_ERR_UNSUPPORTED;
+    prm.scales = scales;
+    prm.y = y;
+    prm.M = M;
+    prm.N = N;
+    prm.K = K;
+    prm.idesc = prefill::make_idesc(decode_tc::kRows, decode_tc::kBatch);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((N + decode_tc::kRows - 1) / decode_tc::kRows, 1, 1);
+    cfg.blockDim = dim3(decode_tc::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = decode_tc::SmemLayout::total;
+    cfg.stream = stream;
+    return cudaLaunchKernelEx(&cfg, decode_tc::decode_tc_kernel, prm) == cudaSuccess ? W3_OK : W3_ERR_CUDA;
 }
 
 w3_status launch_prefill(const uint16_t *x, const int32_t *packed, const uint16_t *scales, uint16_t *y, int M,
@@ -352,6 +396,13 @@ w3_status w3a16_gemm(const uint16_t *x, const int32_t *packed, const uint16_t *s
     // Batches above 16 rows without the tensor-core path run as 16-row decode passes.
     for (int64_t m0 = 0; m0 < M; m0 += 16) {
         const int mb = static_cast<int>(std::min<int64_t>(16, M - m0));
+        // the tensor-core decode walks all of K per 128-row CTA: use it when the rows alone fill the GPU
+        if (mb >= W3_DECODE_TC_MIN_M && (N + decode_tc::kRows - 1) / decode_tc::kRows >= sms) {
+            const w3_status s = launch_decode_tc(x + m0 * K, packed, scales, y + m0 * N, mb, static_cast<int>(N),
+                                                 static_cast<int>(K), st);
+            if (s == W3_OK) continue;
+            if (s != W3_ERR_UNSUPPORTED) return s;
+        }
         const bool sk = W3_DECODE_STREAMK && decode_sk::applicable(mb, static_cast<int>(N), static_cast<int>(K));
         w3_status s = sk ? launch_decode_sk(x + m0 * K, packed, scales, y + m0 * N, mb, static_cast<int>(N),
                                             static_cast<int>(K), sms, st)
