@@ -42,6 +42,7 @@ ROTATE = 5
 WORKLOAD = "Llama-3.1-70B gate_proj N=28672 K=8192, W3A16 g128 decode batch M=1,4,16"
 FALLBACK_HBM_GBS = 6650.0
 DECODE_SOURCES = ("w3a16_gemv_b200/csrc/decode_gemv.cuh", "w3a16_gemv_b200/csrc/decode_streamk.cuh",
+                  "w3a16_gemv_b200/csrc/decode_tcgen05.cuh", "w3a16_gemv_b200/csrc/prefill_gemm.cuh",
                   "w3a16_gemv_b200/csrc/common.cuh")
 
 
@@ -51,10 +52,10 @@ def algorithmic_bytes(M: int, N: int, K: int) -> int:
 
 def kernel_name(M: int) -> str:
     """The kernel w3a16_gemm launches for a decode batch of M rows on the gate_proj shape."""
-    mt = 1 if M <= 1 else 2 if M <= 2 else 4 if M <= 4 else 8 if M <= 8 else 16
-    if mt <= 4:
+    if M <= 4:
+        mt = 1 if M <= 1 else 2 if M <= 2 else 4
         return f"w3::decode_sk::decode_sk_kernel<{mt}> (M={M})"
-    return f"w3::decode::decode_kernel<{mt}> (M={M})"
+    return f"w3::decode_tc::decode_tc_kernel (M={M})"
 
 
 def step_bytes() -> int:

@@ -22,8 +22,11 @@
  *
  * Conventions for every entry point:
  *   - all array pointers are DEVICE pointers (cudaMalloc'd or torch CUDA
- *     tensors) on the current device; the caller owns every buffer and the
- *     library allocates no device memory;
+ *     tensors) on the current device; the caller owns every buffer.  The
+ *     only device memory the library allocates is the scratch of w3a16_gemm
+ *     (at most 32 KB per SM, for partial sums), taken from and returned to a
+ *     private stream-ordered pool on `stream` within the call, so calls on
+ *     different streams never share it;
  *   - bf16 values are passed as their 16-bit patterns (uint16_t);
  *   - every array pointer must be 16-byte aligned (W3_ERR_ALIGN otherwise);
  *   - calls only enqueue work on `stream` (NULL = the legacy default stream)
@@ -105,9 +108,10 @@ w3_status w3_dequant_f32(const int32_t *packed, const uint16_t *scales, float *w
  *   y      [M,N] bf16, row-major; every element is written
  * Arithmetic: fp32 accumulation; the result is rounded once to bf16 (nearest
  * even).  For M <= 16 the weight enters the products exactly (q and the
- * scale are applied in fp32); for M > 16 each weight is first rounded to
- * bf16(q*s) and fed to the tensor cores.  Repeated calls with the same
- * arguments give bit-identical y (no floating-point atomics).
+ * scale are applied in fp32; K may be split over several thread blocks, whose
+ * fp32 partial sums are added in a fixed order); for M > 16 each weight is
+ * first rounded to bf16(q*s) and fed to the tensor cores.  Repeated calls
+ * with the same arguments give bit-identical y (no floating-point atomics).
  * Errors: W3_ERR_NULL, W3_ERR_SHAPE (M, N < 1; K < 128 or K % 128 != 0;
  * M*K, N*K or M*N above 2^40), W3_ERR_ALIGN, W3_ERR_ALIAS (y overlaps x,
  * packed or scales), W3_ERR_UNSUPPORTED, W3_ERR_CUDA.

@@ -40,6 +40,9 @@ SMALL = [
     (12, 300, 1024, "uniform8", "lognormal", "normal"),
     (16, 129, 256, "uniform8", "lognormal", "normal"),
     (16, 1000, 8192, "uniform8", "lognormal", "normal"),
+    (6, 200, 1152, "gsq_uniform", "lognormal", "normal"),         # K split 5 + 4 groups
+    (10, 256, 4224, "uniform8", "absnormal", "normal_outliers"),  # K split 8 ways, last rank idle
+    (13, 28672, 256, "uniform8", "lognormal", "normal"),          # many row tiles, two groups
     (1, 2000, 128, "uniform8", "lognormal", "normal"),
     (1, 64, 28672, "gsq_5level", "absnormal", "normal_outliers"),
     (17, 50, 512, "uniform8", "lognormal", "normal"),

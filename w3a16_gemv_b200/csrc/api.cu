@@ -43,12 +43,13 @@ struct DeviceState {
     std::once_flag once;
     w3_status status = W3_OK;
     int num_sms = 0;
+    cudaMemPool_t pool = nullptr;  // stream-ordered scratch of w3a16_gemm (kept, never trimmed)
 };
 DeviceState g_dev[kMaxDevices];
 
 // Once per device: check that it is an sm_100 part and raise the kernels'
 // dynamic shared-memory limits.
-w3_status device_setup(int *num_sms) {
+w3_status device_setup(int *num_sms, cudaMemPool_t *pool = nullptr) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return W3_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return W3_ERR_UNSUPPORTED;
@@ -90,6 +91,16 @@ w3_status device_setup(int *num_sms) {
             st.status = W3_ERR_CUDA;
             return;
         }
+        cudaMemPoolProps props = {};
+        props.allocType = cudaMemAllocationTypePinned;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = dev;
+        uint64_t keep = UINT64_MAX;
+        if (cudaMemPoolCreate(&st.pool, &props) != cudaSuccess ||
+            cudaMemPoolSetAttribute(st.pool, cudaMemPoolAttrReleaseThreshold, &keep) != cudaSuccess) {
+            st.status = W3_ERR_CUDA;
+            return;
+        }
         if (cudaFuncSetAttribute(prefill::prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  prefill::SmemLayout::total) != cudaSuccess) {
             st.status = W3_ERR_CUDA;
@@ -104,6 +115,7 @@ w3_status device_setup(int *num_sms) {
         st.status = W3_OK;
     });
     *num_sms = st.num_sms;
+    if (pool) *pool = st.pool;
     return st.status;
 }
 
@@ -188,16 +200,23 @@ w3_status launch_decode_sk(const uint16_t *x, const int32_t *packed, const uint1
     return e == cudaSuccess ? W3_OK : W3_ERR_CUDA;
 }
 
-// Tensor-core decode (tcgen05, weights as the MMA's M dimension).  Returns
-// W3_ERR_UNSUPPORTED, without launching, when a tensor map for this shape
-// cannot be encoded; the caller then uses the mma.sync kernels.
+// Tensor-core decode (tcgen05, weights as the MMA's M dimension), M <= 16.
+// Shared tiles are finished by the fix-up kernel, launched behind it with
+// programmatic dependent launch; their fp32 partial sums live in `partial`
+// (decode_tc::plan(...).ws_floats floats, unused when that is 0).  Returns
+// W3_ERR_UNSUPPORTED, without launching, for shapes it does not take (N < 256).
 w3_status launch_decode_tc(const uint16_t *x, const int32_t *packed, const uint16_t *scales, uint16_t *y, int M,
-                           int N, int K, cudaStream_t stream) {
+                           int N, int K, const decode_tc::LaunchPlan &P, float *partial, cudaStream_t stream) {
+    if (N < decode_tc::kRows || M > decode_tc::kBatch) return W3_ERR_UNSUPPORTED;
     decode_tc::Params prm;
     const int64_t words = static_cast<int64_t>(K) * 3 / 32;
-    if (N < decode_tc::kRows || words < decode_tc::kPitch) return W3_ERR_UNSUPPORTED;
-    if (encode_packed_map(&prm.tmap_w, packed, N, words, decode_tc::kPitch, decode_tc::kRows) != W3_OK)
-        return W3_ERR_UNSUPPORTED;
+    if (encode_packed_map(&prm.tmap_w1, packed, N, words, decode_tc::kPitch1, decode_tc::kRows) != W3_OK)
+        return W3_ERR_CUDA;
+    prm.has_w3 = words >= decode_tc::kPitch3;
+    prm.tmap_w3 = prm.tmap_w1;
+    if (prm.has_w3 &&
+        encode_packed_map(&prm.tmap_w3, packed, N, words, decode_tc::kPitch3, decode_tc::kRows) != W3_OK)
+        return W3_ERR_CUDA;
     PFN_cuTensorMapEncodeTiled enc = tensor_map_encoder();
     if (!enc) return W3_ERR_CUDA;
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
@@ -207,19 +226,42 @@ w3_status launch_decode_tc(const uint16_t *x, const int32_t *packed, const uint1
     if (enc(&prm.tmap_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t *>(x), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return W3_ERR_UNSUPPORTED;
+        return W3_ERR_CUDA;
     prm.scales = scales;
     prm.y = y;
+    prm.partial = partial;
     prm.M = M;
     prm.N = N;
     prm.K = K;
-    prm.idesc = prefill::make_idesc(decode_tc::kRows, decode_tc::kBatch);
+    prm.G = K / kGroup;
+    prm.P = P.P;
+    prm.U = P.U;
+    prm.idesc = prefill::make_idesc(decode_tc::kTileRows, decode_tc::kBatch);
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((N + decode_tc::kRows - 1) / decode_tc::kRows, 1, 1);
+    cfg.gridDim = dim3(P.P, 1, 1);
     cfg.blockDim = dim3(decode_tc::kThreads, 1, 1);
     cfg.dynamicSmemBytes = decode_tc::SmemLayout::total;
     cfg.stream = stream;
-    return cudaLaunchKernelEx(&cfg, decode_tc::decode_tc_kernel, prm) == cudaSuccess ? W3_OK : W3_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, decode_tc::decode_tc_kernel, prm) != cudaSuccess) return W3_ERR_CUDA;
+    if (P.P == 1) return W3_OK;
+    decode_tc::FixupParams fp;
+    fp.partial = partial;
+    fp.y = y;
+    fp.M = M;
+    fp.N = N;
+    fp.G = prm.G;
+    fp.P = P.P;
+    fp.U = P.U;
+    cudaLaunchConfig_t fcfg = {};
+    fcfg.gridDim = dim3(P.P - 1, 1, 1);
+    fcfg.blockDim = dim3(decode_tc::kRows, 1, 1);
+    fcfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    fcfg.attrs = attr;
+    fcfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&fcfg, decode_tc::decode_tc_fixup_kernel, fp) == cudaSuccess ? W3_OK : W3_ERR_CUDA;
 }
 
 w3_status launch_prefill(const uint16_t *x, const int32_t *packed, const uint16_t *scales, uint16_t *y, int M,
@@ -388,29 +430,40 @@ w3_status w3a16_gemm(const uint16_t *x, const int32_t *packed, const uint16_t *s
         overlaps(y, ybytes, scales, N * (K / kGroup) * 2))
         return W3_ERR_ALIAS;
     int sms;
-    if (w3_status s = device_setup(&sms)) return s;
+    cudaMemPool_t pool;
+    if (w3_status s = device_setup(&sms, &pool)) return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (M > 16 && W3_PREFILL_TCGEN05)
         return launch_prefill(x, packed, scales, y, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), sms,
                               st);
+    // The tensor-core decode for N >= 256: one call per 16 batch rows, all sharing
+    // one stream-ordered scratch buffer for the partial sums.
+    const bool tc = N >= decode_tc::kRows && W3_DECODE_TC_MIN_M <= std::min<int64_t>(M, 16);
+    const decode_tc::LaunchPlan tplan = decode_tc::plan(N, K, sms);
+    float *partial = nullptr;
+    if (tc && tplan.ws_floats > 0 &&
+        cudaMallocFromPoolAsync(reinterpret_cast<void **>(&partial), tplan.ws_floats * sizeof(float), pool, st) !=
+            cudaSuccess)
+        return W3_ERR_CUDA;
+    w3_status status = W3_OK;
     // Batches above 16 rows without the tensor-core path run as 16-row decode passes.
-    for (int64_t m0 = 0; m0 < M; m0 += 16) {
+    for (int64_t m0 = 0; m0 < M && status == W3_OK; m0 += 16) {
         const int mb = static_cast<int>(std::min<int64_t>(16, M - m0));
-        // the tensor-core decode walks all of K per 128-row CTA: use it when the rows alone fill the GPU
-        if (mb >= W3_DECODE_TC_MIN_M && (N + decode_tc::kRows - 1) / decode_tc::kRows >= sms) {
-            const w3_status s = launch_decode_tc(x + m0 * K, packed, scales, y + m0 * N, mb, static_cast<int>(N),
-                                                 static_cast<int>(K), st);
-            if (s == W3_OK) continue;
-            if (s != W3_ERR_UNSUPPORTED) return s;
+        if (tc && mb >= W3_DECODE_TC_MIN_M) {
+            status = launch_decode_tc(x + m0 * K, packed, scales, y + m0 * N, mb, static_cast<int>(N),
+                                      static_cast<int>(K), tplan, partial, st);
+            if (status == W3_OK) continue;
+            if (status != W3_ERR_UNSUPPORTED) break;
+            status = W3_OK;
         }
         const bool sk = W3_DECODE_STREAMK && decode_sk::applicable(mb, static_cast<int>(N), static_cast<int>(K));
-        w3_status s = sk ? launch_decode_sk(x + m0 * K, packed, scales, y + m0 * N, mb, static_cast<int>(N),
-                                            static_cast<int>(K), sms, st)
-                         : launch_decode(x + m0 * K, packed, scales, y + m0 * N, mb, static_cast<int>(N),
-                                         static_cast<int>(K), sms, st);
-        if (s) return s;
+        status = sk ? launch_decode_sk(x + m0 * K, packed, scales, y + m0 * N, mb, static_cast<int>(N),
+                                       static_cast<int>(K), sms, st)
+                    : launch_decode(x + m0 * K, packed, scales, y + m0 * N, mb, static_cast<int>(N),
+                                    static_cast<int>(K), sms, st);
     }
-    return W3_OK;
+    if (partial && cudaFreeAsync(partial, st) != cudaSuccess && status == W3_OK) status = W3_ERR_CUDA;
+    return status;
 }
 
 w3_status w3_check_device_error(w3_stream_t stream) {

@@ -23,8 +23,10 @@ constexpr int kBytesPerGroup = 48;
 
 // Device error flag bits (read and cleared by w3_check_device_error).
 constexpr unsigned kDevErrTimeout = 1u;
-// A bounded wait gives up after this long (ns of %globaltimer).
-constexpr unsigned long long kWaitLimitNs = 1000000000ull;
+// A bounded wait gives up after this many SM clock cycles (about 2 s at the
+// B200's 1.965 GHz maximum; the SM cycle counter is cheap to read, unlike the
+// global timer).
+constexpr long long kWaitLimitCycles = 4000000000ll;
 
 // Set by kernels, read and cleared by w3_check_device_error (the library is one
 // translation unit, so this is its only definition).
@@ -61,6 +63,15 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
 
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
+#if defined(W3_WAIT_TEST)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+#else
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
@@ -68,17 +79,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         : "=r"(ok)
         : "r"(bar), "r"(parity)
         : "memory");
+#endif
     return ok != 0;
 }
 
-// Wait for phase `parity` of the barrier to complete; give up after kWaitLimitNs,
-// record kDevErrTimeout and return false.
+// Wait for phase `parity` of the barrier to complete; give up after
+// kWaitLimitCycles, record kDevErrTimeout and return false.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;
-    const unsigned long long t0 = globaltimer_ns();
+    const long long t0 = clock64();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        if (clock64() - t0 > kWaitLimitCycles) {
             record_error(kDevErrTimeout);
             return false;
         }

@@ -3,33 +3,50 @@
 // model card ("Storage layout" section), never materialised in memory.
 //
 // The roles of the operands are swapped with respect to a GEMM over the batch:
-// the weights are the MMA's M dimension (128 rows per CTA) and the batch is
-// its N dimension (16 columns, rows of x beyond M read as zeros).
+// the weights are the MMA's M dimension (two 128-row tiles per CTA) and the
+// batch is its N dimension (16 columns; rows of x beyond M read as zeros and
+// their columns of the result are never stored).  The unpack of a weight is
+// done once whatever M is, and the tensor cores do all of the multiply-adds.
 //
-//  * Loads: one warp issues, per stage of 3 groups, one tiled TMA copy of the
-//    packed words of the CTA's 128 rows ([128 rows][36 words]) and six copies
-//    of x ([16 rows][64 k], 128-byte swizzle, the UMMA B-operand layout).
-//  * Row warps (4 x 32 threads, one weight row per thread): for each group the
-//    thread reads its row's 12 words, expands the 128 codes in natural k order
-//    to the exact levels q = c - 4 in bf16 (12 bits of two code pairs times
-//    0x2001 put each pair's second code 13 bits above its first; one LOP3 per
-//    pair into the mantissa of bf16 128.0, then a bf16x2 subtract of 132), and
-//    writes the 64 bf16x2 words into its tensor-memory lane with one
-//    tcgen05.st -- the A operand, double-buffered.
-//  * One thread issues 8 tcgen05.mma (A from tensor memory, B = x from shared
-//    memory, fp32 accumulation in tensor memory) per group into a fresh
-//    per-group accumulator of 16 columns.
-//  * The row threads read each group's 16 results back (tcgen05.ld) and add
-//    s[n,g] * D to fp32 registers: the group scale is applied in fp32 and
-//    nothing is rounded before the final bf16 store.
+//  * Work: the (256-row tile, group) units of the matrix are split into equal
+//    contiguous ranges, one per CTA and one CTA per SM (stream-K).  A range
+//    covers the end of one tile, whole tiles and the start of another; a tile
+//    that several CTAs share is finished by a small second kernel that adds
+//    their fp32 partial sums in CTA order, so the result does not depend on
+//    timing.
+//  * Loads (one warp): per stage of up to 3 groups, one tiled TMA copy of the
+//    packed words of the CTA's 256 rows ([256 rows][36 words], or one
+//    [256 rows][12 words] copy per group) and two copies of x per group
+//    ([16 rows][64 k], 128-byte swizzle: the UMMA B-operand layout).  The same
+//    warp then permutes each 32-k block of x in place into the order of the
+//    unpack below (byte permutes, no arithmetic).  A second warp copies the
+//    stage's group scales (256 rows x up to 3) into a shared-memory ring, so
+//    no row thread ever waits on a global load.
+//  * Row warps (8 x 32 threads, one weight row per thread): a 32-code block
+//    (3 words) becomes 16 bf16x2 words with 16 LOP3s and 9 shifts -- the same
+//    pair schedule as the mma.sync decode: each LOP3 drops two codes into the
+//    mantissa of bf16 128.0 at bit offsets e_lo, e_hi, the exact value
+//    128 + c*2^e -- and one bf16x2 FMA per pair, v*2^-e - (128*2^-e + 4),
+//    turns each into the exact level q = c - 4.  The 64 words of a group go
+//    to the thread's tensor-memory lane with one tcgen05.st: the A operand,
+//    three group buffers per tile.
+//  * One thread issues 8 tcgen05.mma per group and tile (A from tensor memory,
+//    B = permuted x from shared memory) into a fresh per-group fp32
+//    accumulator of 16 columns (four buffers per tile).
+//  * The row threads read each group's 16 results back two groups later
+//    (tcgen05.ld) and add s[n,g] * D to fp32 registers: the group scale is
+//    applied in fp32 and nothing is rounded before the final bf16 store.
 #pragma once
 
 #include "common.cuh"
+#include "decode_gemv.cuh"
 #include "prefill_gemm.cuh"
 
 namespace w3 {
 namespace decode_tc {
 
+using decode::pair_spec;
+using prefill::desc_add;
 using prefill::fence_async_smem;
 using prefill::mbar_arrive;
 using prefill::sw128_kmajor_desc;
@@ -37,46 +54,118 @@ using prefill::tc_fence_after;
 using prefill::tc_fence_before;
 using prefill::umma_commit;
 
-constexpr int kRows = 128;             // weight rows per CTA = UMMA M
-constexpr int kBatch = 16;             // UMMA N: batch rows (x rows >= M are zero)
+constexpr int kTileRows = 128;                    // UMMA M: one tensor-memory lane per row
+constexpr int kTiles = 2;                         // row tiles per CTA, sharing x
+constexpr int kRows = kTiles * kTileRows;         // 256 rows per CTA (one TMA box)
+constexpr int kBatch = 16;                        // UMMA N
 constexpr int kStageGroups = 3;
-constexpr int kStages = 3;
-constexpr int kPitch = kStageGroups * kWordsPerGroup;       // 36 words per row and stage
-constexpr int kPackedBytes = kRows * kPitch * 4;            // 18432
-constexpr int kXBox = kBatch * 64 * 2;                      // 2 KB: [16 rows][64 k] bf16
-constexpr int kXBytes = kStageGroups * 2 * kXBox;           // 12 KB per stage
-constexpr int kABuffers = 2, kDBuffers = 2;
-constexpr int kAColsPerGroup = kGroup / 2;                  // 64 columns: two bf16 per column
-constexpr int kTmemCols = 256;
-constexpr int kThreads = 6 * 32;                            // TMA warp, MMA warp, 4 row warps
-static_assert(kPackedBytes % 1024 == 0 && kXBytes % 1024 == 0, "stage buffers keep 1024-byte alignment");
+constexpr int kStages = 4;
+constexpr int kPitch3 = kStageGroups * kWordsPerGroup;        // 36 words: rows of a 3-group box
+constexpr int kPitch1 = kWordsPerGroup;                       // 12 words: rows of a 1-group box
+constexpr int kBox1Bytes = kRows * kPitch1 * 4;               // 12 KB
+constexpr int kXBox = kBatch * 64 * 2;                        // 2 KB: [16 rows][64 k] bf16
+constexpr int kXGroupBytes = 2 * kXBox;                       // 4 KB
+constexpr int kXBytes = kStageGroups * kXGroupBytes;          // 12 KB
+constexpr int kStageBytes = kXBytes + kStageGroups * kBox1Bytes;  // 48 KB
+constexpr int kABuf = 3;                                      // A buffers (one group each) per tile
+constexpr int kDBuf = 4;                                      // accumulators per tile
+constexpr int kLag = 2;                                       // groups between MMA and read-back
+constexpr int kACols = 64;                                    // 128 codes, two bf16 per column
+constexpr int kDCol0 = kABuf * kACols;                        // 192
+constexpr int kTileCols = kDCol0 + kDBuf * kBatch;            // 256 columns per tile
+constexpr int kTmemCols = kTiles * kTileCols;                 // 512: one CTA per SM
+constexpr int kRowWarps = kTiles * 4;
+constexpr int kScaleWarp = 2 + kRowWarps;                     // warp 10
+constexpr int kThreads = (3 + kRowWarps) * 32;                // load, MMA, row warps, scale warp
+constexpr int kScaleSlotBytes = kStageGroups * kRows * 2;     // [3 groups][256 rows] bf16
+#ifndef W3_DECODE_TC_MIN_UNITS
+#define W3_DECODE_TC_MIN_UNITS 6
+#endif
+constexpr int kMinUnitsPerCta = W3_DECODE_TC_MIN_UNITS;
+static_assert(kXGroupBytes % 1024 == 0 && kXBytes % 1024 == 0 && kStageBytes % 1024 == 0,
+              "swizzled x boxes need 1024-byte alignment");
+static_assert(kBox1Bytes % 128 == 0, "tiled TMA destinations need 128-byte alignment");
+static_assert(kStageGroups * kBox1Bytes == kRows * kPitch3 * 4, "a 3-group box fills the same bytes");
+// The row threads read group j - kDBuf back (iteration j - kDBuf + kLag) before they
+// hand over the A operand of group j, so "A of group j is full" also means "the
+// accumulator of group j is free" and the MMA side needs no separate barrier.
+static_assert(kDBuf >= kLag + 1, "read-back must finish before the accumulator is reused");
 
 struct SmemLayout {
-    static constexpr int x_off = 0;                                    // [kStages][kXBytes], 1024-aligned
-    static constexpr int packed_off = x_off + kStages * kXBytes;       // [kStages][kPackedBytes]
-    static constexpr int bar_off = packed_off + kStages * kPackedBytes;
-    // stage_full, stage_empty [kStages]; a_full, a_free [kABuffers]; d_full, d_free [kDBuffers]
-    static constexpr int nbars = 2 * kStages + 2 * kABuffers + 2 * kDBuffers;
+    static constexpr int stage_off = 0;  // [kStages]{x: [3][2 boxes], packed}
+    static constexpr int scale_off = stage_off + kStages * kStageBytes;  // [kStages][3][256] bf16
+    static constexpr int bar_off = scale_off + kStages * kScaleSlotBytes;
+    // full, empty, bready [kStages]; a_full [kTiles][kABuf]; done [kTiles][kDBuf] (the MMAs of a group)
+    static constexpr int nbars = 3 * kStages + kTiles * kABuf + kTiles * kDBuf;
     static constexpr int tmem_slot_off = bar_off + nbars * 8;
-    static constexpr int total = tmem_slot_off + 16 + 1024;
+    static constexpr int total = tmem_slot_off + 16 + 1024;  // + slack for 1024-byte alignment
 };
+static_assert(SmemLayout::total <= 227 * 1024, "shared memory per CTA");
 
 struct Params {
-    CUtensorMap tmap_w;  // packed [N][3K/32] u32, box [128 rows][36 words]
-    CUtensorMap tmap_x;  // x [M][K] bf16, box [16 rows][64 k], 128-byte swizzle
+    CUtensorMap tmap_w3;  // packed [N][3K/32] u32, box [256 rows][36 words] (valid when has_w3)
+    CUtensorMap tmap_w1;  // packed, box [256 rows][12 words]
+    CUtensorMap tmap_x;   // x [M][K] bf16, box [16 rows][64 k], 128-byte swizzle
     const uint16_t *scales;
     uint16_t *y;
+    float *partial;       // [P][2][16][256] fp32 partial sums of shared tiles
     int M, N, K;
-    uint32_t idesc;      // UMMA M=128, N=16, bf16 x bf16 -> f32
+    int G;                // groups per row
+    int P;                // CTAs
+    int has_w3;
+    int64_t U;            // units: 256-row tiles x groups
+    uint32_t idesc;       // UMMA M=128, N=16, bf16 x bf16 -> f32
 };
 
-__device__ __forceinline__ void umma_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
-                                        uint32_t accumulate) {
+struct FixupParams {
+    const float *partial;
+    uint16_t *y;
+    int M, N, G, P;
+    int64_t U;
+};
+
+// First unit of CTA c: the ranges [unit_begin(c), unit_begin(c + 1)) tile the units.
+__host__ __device__ inline int64_t unit_begin(int c, int64_t U, int P) { return static_cast<int64_t>(c) * U / P; }
+
+// ---- compile-time constants of the pair schedule ----------------------------------
+
+// bf16 bits of a positive integer v < 256 with at most 8 significant bits.
+__host__ __device__ constexpr uint32_t bf16_of_int(int v) {
+    int e = 0;
+    while ((v >> (e + 1)) != 0) ++e;
+    return static_cast<uint32_t>(((127 + e) << 7) | (((v - (1 << e)) << 7) >> e));
+}
+// bf16x2 (2^-e_lo, 2^-e_hi) and (-(128*2^-e_lo + 4), -(128*2^-e_hi + 4)) for pair i.
+__host__ __device__ constexpr uint32_t pair_mul(int i) {
+    return static_cast<uint32_t>((127 - pair_spec(i).elo) << 7) | (static_cast<uint32_t>(127 - pair_spec(i).ehi) << 23);
+}
+__host__ __device__ constexpr uint32_t pair_add(int i) {
+    return (0x8000u | bf16_of_int((128 >> pair_spec(i).elo) + 4)) |
+           ((0x8000u | bf16_of_int((128 >> pair_spec(i).ehi) + 4)) << 16);
+}
+static_assert(bf16_of_int(132) == 0x4304u && bf16_of_int(12) == 0x4140u && bf16_of_int(68) == 0x4288u,
+              "bf16 encoding of the level offsets");
+// __byte_perm selector taking element lo of word a and element hi of word b.
+__host__ __device__ constexpr uint32_t pair_sel(int i) {
+    const uint32_t b0 = 2u * (pair_spec(i).lo & 1), b2 = 4u + 2u * (pair_spec(i).hi & 1);
+    return b0 | ((b0 + 1) << 4) | (b2 << 8) | ((b2 + 1) << 12);
+}
+
+__device__ __forceinline__ uint32_t bf16x2_fma(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+// tcgen05.mma with A in tensor memory, called by every lane of a converged
+// warp and issued by one elected lane (see umma_bf16).  ACC: add to D.
+template <bool ACC>
+__device__ __forceinline__ void umma_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc) {
     asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
-        "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        "{\n\t.reg .pred e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, %4;\n\t}" ::"r"(tmem_d),
+        "r"(tmem_a), "l"(bdesc), "r"(idesc), "n"(ACC ? 1 : 0)
         : "memory");
 }
 
@@ -107,64 +196,94 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-// Bits [12q, 12q+12) of a group's 384-bit stream w[0..11]: codes 4q..4q+3.
-template <int Q>
-__device__ __forceinline__ uint32_t quad12(const uint32_t (&w)[12]) {
-    constexpr int b = 12 * Q, i = b / 32, s = b % 32;
-    if constexpr (s + 12 <= 32) return (w[i] >> s) & 0xFFFu;
-    else return __funnelshift_r(w[i], w[i + 1], s) & 0xFFFu;
-}
-
-__device__ __forceinline__ uint32_t bf16x2_sub(uint32_t v, uint32_t sub) {
-    uint32_t q;
-    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(q) : "r"(v), "r"(sub));
-    return q;
-}
-
-// The group's 128 codes as 64 bf16x2 words of exact levels q = c - 4, natural k order.
-template <int Q>
-__device__ __forceinline__ void expand_levels(const uint32_t (&w)[12], uint32_t (&out)[64]) {
-    if constexpr (Q < 32) {
-        constexpr uint32_t kMagic2 = 0x43004300u;  // bf16x2 (128, 128)
-        constexpr uint32_t kSub = 0x43044304u;     // bf16x2 (132, 132)
-        const uint32_t x = quad12<Q>(w) * 0x2001u;
-        out[2 * Q] = bf16x2_sub(and_or<0x00070007u>(x, kMagic2), kSub);
-        out[2 * Q + 1] = bf16x2_sub(and_or<0x00070007u>(x >> 6, kMagic2), kSub);
-        expand_levels<Q + 1>(w, out);
+// A group's 128 codes (12 words) as 64 bf16x2 words of exact levels, in pair order:
+// word 16*b + i holds codes (lo_i, hi_i) of block b.
+__device__ __forceinline__ void group_levels(const uint32_t (&w)[kWordsPerGroup], uint32_t (&a)[64]) {
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+        uint32_t blk[16];
+        decode::unpack_block(w[3 * b], w[3 * b + 1], w[3 * b + 2], blk);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) a[16 * b + i] = bf16x2_fma(blk[i], pair_mul(i), pair_add(i));
     }
 }
 
-__global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(const __grid_constant__ Params p) {
+// Permute x of one stage in place: each 32-k block of each batch row is put in
+// pair order (word i of the block = elements lo_i, hi_i).  The boxes are in the
+// 128-byte swizzle: 16-byte chunk c of row r sits at chunk c ^ (r % 8), so a
+// block's four chunks stay together.
+__device__ __forceinline__ void permute_x(uint8_t *xs, int ns, int lane) {
+    for (int jj = 0; jj < ns; ++jj) {
+#pragma unroll
+        for (int it = 0; it < 2; ++it) {
+            const int item = lane + 32 * it;  // 16 rows x 4 blocks
+            const int r = item & 15, bl = item >> 4;
+            uint8_t *row = xs + jj * kXGroupBytes + (bl >> 1) * kXBox + r * 128;
+            const int h = bl & 1, sw = r & 7;
+            uint32_t src[16];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const uint4 q = *reinterpret_cast<const uint4 *>(row + (((4 * h + c) ^ sw) << 4));
+                src[4 * c] = q.x;
+                src[4 * c + 1] = q.y;
+                src[4 * c + 2] = q.z;
+                src[4 * c + 3] = q.w;
+            }
+            uint32_t out[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                out[i] = __byte_perm(src[pair_spec(i).lo >> 1], src[pair_spec(i).hi >> 1], pair_sel(i));
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                *reinterpret_cast<uint4 *>(row + (((4 * h + c) ^ sw) << 4)) =
+                    make_uint4(out[4 * c], out[4 * c + 1], out[4 * c + 2], out[4 * c + 3]);
+        }
+    }
+}
+
+// Walks a CTA's unit range as segments (one per 256-row tile touched); every
+// role walks the same segments and splits them into the same stages.
+struct Walk {
+    int64_t u, end;
+    int G;
+    __device__ explicit Walk(const Params &p)
+        : u(unit_begin(blockIdx.x, p.U, p.P)), end(unit_begin(blockIdx.x + 1, p.U, p.P)), G(p.G) {}
+    // next segment: tile t, first group g0, length len; false when done
+    __device__ bool next(int64_t &t, int &g0, int &len) {
+        if (u >= end) return false;
+        t = u / G;
+        g0 = static_cast<int>(u - t * G);
+        const int64_t se = (t + 1) * G < end ? (t + 1) * G : end;
+        len = static_cast<int>(se - u);
+        u = se;
+        return true;
+    }
+};
+
+__global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_constant__ Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_addr(smem);
-    const uint32_t x_base = sbase + SmemLayout::x_off;
-    const uint32_t w_base = sbase + SmemLayout::packed_off;
     const uint32_t bars = sbase + SmemLayout::bar_off;
-    const uint32_t stage_full = bars, stage_empty = bars + 8 * kStages;
-    const uint32_t a_full = bars + 16 * kStages, a_free = a_full + 8 * kABuffers;
-    const uint32_t d_full = a_free + 8 * kABuffers, d_free = d_full + 8 * kDBuffers;
+    const uint32_t bar_full = bars, bar_empty = bars + 8 * kStages, bar_bready = bars + 16 * kStages;
+    const uint32_t bar_afull = bars + 24 * kStages;                // [kTiles][kABuf]
+    const uint32_t bar_done = bar_afull + 8 * kTiles * kABuf;      // [kTiles][kDBuf]
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + SmemLayout::tmem_slot_off);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int n0 = blockIdx.x * kRows;
-    const int G = p.K / kGroup;
-    const int nstages = (G + kStageGroups - 1) / kStageGroups;
+
+    // the partial-sum fix-up grid may start now; it waits for this grid to finish
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(stage_full + 8 * s, 1);
-            mbar_init(stage_empty + 8 * s, kRows + 1);  // row threads read the words, the MMAs read x
+            mbar_init(bar_full + 8 * s, 1 + 32);  // the TMA bytes and the 32 lanes of the scale warp
+            mbar_init(bar_empty + 8 * s, kRows + 1);  // row threads read the words, the MMAs read x
+            mbar_init(bar_bready + 8 * s, 1);
         }
-        for (int b = 0; b < kABuffers; ++b) {
-            mbar_init(a_full + 8 * b, kRows);
-            mbar_init(a_free + 8 * b, 1);
-        }
-        for (int b = 0; b < kDBuffers; ++b) {
-            mbar_init(d_full + 8 * b, 1);
-            mbar_init(d_free + 8 * b, kRows);
-        }
+        for (int b = 0; b < kTiles * kABuf; ++b) mbar_init(bar_afull + 8 * b, kTileRows);
+        for (int b = 0; b < kTiles * kDBuf; ++b) mbar_init(bar_done + 8 * b, 1);
         mbar_init_fence();
     }
     if (warp == 1) {
@@ -177,105 +296,211 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(const __grid_con
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tmem_a = tmem;                                   // [kABuffers][64 columns]
-    const uint32_t tmem_d = tmem + kABuffers * kAColsPerGroup;      // [kDBuffers][16 columns]
     bool ok = true;
 
     if (warp == 0) {
-        if (lane == 0) {  // ---- loads ----
-            for (int s = 0; s < nstages && ok; ++s) {
-                const int slot = s % kStages;
-                ok = mbar_wait_bounded(stage_empty + 8 * slot, ((s / kStages) & 1) ^ 1);
+        // ---- loads, then the in-place permutation of x one stage behind ----
+        Walk walk(p);
+        int64_t t;
+        int g0, len, stage = 0, prev_ns = 0;
+        auto prep = [&](int st, int ns) {
+            const int slot = st % kStages;
+            ok = ok && __all_sync(0xffffffffu, mbar_wait_bounded(bar_full + 8 * slot, (st / kStages) & 1));
+            if (!ok) return;
+            permute_x(smem + SmemLayout::stage_off + slot * kStageBytes, ns, lane);
+            fence_async_smem();  // generic writes -> read by the tensor cores (async proxy)
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_bready + 8 * slot);
+        };
+        while (ok && walk.next(t, g0, len)) {
+            for (int gs = 0; gs < len && ok; gs += kStageGroups) {
+                const int ns = min(kStageGroups, len - gs);
+                const int slot = stage % kStages;
+                if (lane == 0) {
+                    ok = mbar_wait_bounded(bar_empty + 8 * slot, ((stage / kStages) & 1) ^ 1);
+                    if (ok) {
+                        const uint32_t bar = bar_full + 8 * slot;
+                        const uint32_t st = sbase + SmemLayout::stage_off + slot * kStageBytes;
+                        const int g = g0 + gs;
+                        const int row0 = static_cast<int>(t * kRows);
+                        mbar_arrive_expect_tx(bar, ns * (kXGroupBytes + kBox1Bytes));
+                        for (int jj = 0; jj < ns; ++jj) {
+                            tma_load_2d(st + jj * kXGroupBytes, &p.tmap_x, (g + jj) * kGroup, 0, bar);
+                            tma_load_2d(st + jj * kXGroupBytes + kXBox, &p.tmap_x, (g + jj) * kGroup + 64, 0, bar);
+                        }
+                        if (ns == kStageGroups && p.has_w3) {
+                            tma_load_2d(st + kXBytes, &p.tmap_w3, g * kWordsPerGroup, row0, bar);
+                        } else {
+                            for (int jj = 0; jj < ns; ++jj)
+                                tma_load_2d(st + kXBytes + jj * kBox1Bytes, &p.tmap_w1, (g + jj) * kWordsPerGroup,
+                                            row0, bar);
+                        }
+                    }
+                }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) break;
-                const uint32_t bar = stage_full + 8 * slot;
-                mbar_arrive_expect_tx(bar, kPackedBytes + kXBytes);
-                tma_load_2d(w_base + slot * kPackedBytes, &p.tmap_w, s * kPitch, n0, bar);
-                const uint32_t xs = x_base + slot * kXBytes;
-#pragma unroll
-                for (int h = 0; h < 2 * kStageGroups; ++h)
-                    tma_load_2d(xs + h * kXBox, &p.tmap_x, (s * kStageGroups * 2 + h) * 64, 0, bar);
+                if (stage > 0) prep(stage - 1, prev_ns);
+                prev_ns = ns;
+                ++stage;
             }
         }
+        if (ok && stage > 0) prep(stage - 1, prev_ns);
     } else if (warp == 1) {
-        if (lane == 0) {  // ---- MMA issue ----
-            for (int j = 0; j < G && ok; ++j) {
-                const int s = j / kStageGroups, gi = j % kStageGroups, slot = s % kStages;
-                const int ab = j % kABuffers, db = j % kDBuffers;
-                if (gi == 0) ok = mbar_wait_bounded(stage_full + 8 * slot, (s / kStages) & 1);
-                ok = ok && mbar_wait_bounded(a_full + 8 * ab, (j / kABuffers) & 1) &&
-                     mbar_wait_bounded(d_free + 8 * db, ((j / kDBuffers) & 1) ^ 1);
-                if (!ok) break;
-                tc_fence_after();
-                const uint32_t xg = x_base + slot * kXBytes + gi * 2 * kXBox;
+        // ---- MMA issue: per group and tile, 8 MMAs into a fresh accumulator; the
+        //      whole warp runs the loop and one elected lane issues ----
+        Walk walk(p);
+        int64_t t;
+        int g0, len, stage = 0, j = 0;
+        const uint64_t xdesc0 = sw128_kmajor_desc(sbase + SmemLayout::stage_off);
+        while (ok && walk.next(t, g0, len)) {
+            for (int gs = 0; gs < len && ok; gs += kStageGroups) {
+                const int ns = min(kStageGroups, len - gs);
+                const int slot = stage % kStages;
+                ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar_bready + 8 * slot, (stage / kStages) & 1));
+                const uint64_t xd = desc_add(xdesc0, slot * kStageBytes);
+                for (int jj = 0; jj < ns && ok; ++jj, ++j) {
+                    const int ab = j % kABuf, db = j % kDBuf;
+                    for (int tile = 0; tile < kTiles && ok; ++tile) {
+                        ok = __all_sync(0xffffffffu,
+                                        mbar_wait_bounded(bar_afull + 8 * (tile * kABuf + ab), (j / kABuf) & 1));
+                        if (!ok) break;
+                        tc_fence_after();
+                        const uint32_t tt = tmem + tile * kTileCols;
+                        const uint32_t dcol = tt + kDCol0 + db * kBatch, acol = tt + ab * kACols;
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    umma_ts(tmem_d + db * kBatch, tmem_a + ab * kAColsPerGroup + kk * 8,
-                            sw128_kmajor_desc(xg + (kk / 4) * kXBox + (kk % 4) * 32), p.idesc, kk > 0 ? 1u : 0u);
-                umma_commit(a_free + 8 * ab);
-                umma_commit(d_full + 8 * db);
-                if (gi == kStageGroups - 1 || j == G - 1) umma_commit(stage_empty + 8 * slot);
+                        for (int kk = 0; kk < 8; ++kk) {
+                            const uint64_t bd = desc_add(xd, jj * kXGroupBytes + (kk >> 2) * kXBox + (kk & 3) * 32);
+                            if (kk == 0) umma_ts<false>(dcol, acol, bd, p.idesc);
+                            else umma_ts<true>(dcol, acol + kk * 8, bd, p.idesc);
+                        }
+                        umma_commit(bar_done + 8 * (tile * kDBuf + db));  // A read, D written
+                    }
+                }
+                if (!ok) break;
+                umma_commit(bar_empty + 8 * slot);
+                ++stage;
+            }
+        }
+    } else if (warp == kScaleWarp) {
+        // ---- group scales of each stage into the shared-memory ring ----
+        Walk walk(p);
+        int64_t t;
+        int g0, len, stage = 0;
+        while (ok && walk.next(t, g0, len)) {
+            for (int gs = 0; gs < len && ok; gs += kStageGroups) {
+                const int ns = min(kStageGroups, len - gs);
+                const int slot = stage % kStages;
+                ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar_empty + 8 * slot, ((stage / kStages) & 1) ^ 1));
+                if (!ok) break;
+                uint16_t *dst = reinterpret_cast<uint16_t *>(smem + SmemLayout::scale_off + slot * kScaleSlotBytes);
+                uint16_t v[kRows / 32][kStageGroups];
+#pragma unroll
+                for (int q = 0; q < kRows / 32; ++q) {
+                    const int64_t n = t * kRows + lane + 32 * q;
+                    const uint16_t *src = p.scales + (n < p.N ? n : p.N - 1) * static_cast<int64_t>(p.G) + g0 + gs;
+#pragma unroll
+                    for (int jj = 0; jj < kStageGroups; ++jj) v[q][jj] = jj < ns ? __ldg(src + jj) : uint16_t(0);
+                }
+#pragma unroll
+                for (int q = 0; q < kRows / 32; ++q)
+#pragma unroll
+                    for (int jj = 0; jj < kStageGroups; ++jj) dst[jj * kRows + lane + 32 * q] = v[q][jj];
+                mbar_arrive(bar_full + 8 * slot);  // release: the stores above are visible to the waiters
+                ++stage;
             }
         }
     } else {
         // ---- row warps: one weight row per thread ----
-        const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
-        const int r = quarter * 32 + lane;
-        const int n = n0 + r;
-        const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-        const uint16_t *srow = p.scales + static_cast<int64_t>(min(n, p.N - 1)) * G;
+        const int tile = (warp - 2) >> 2;
+        const int quarter = warp & 3;  // a warp reaches TMEM lanes 32*(warp % 4) .. +31
+        const int r = tile * kTileRows + quarter * 32 + lane;
+        const uint32_t tt = tmem + tile * kTileCols + (static_cast<uint32_t>(quarter * 32) << 16);
+        const uint32_t afull = bar_afull + 8 * tile * kABuf, done = bar_done + 8 * tile * kDBuf;
         float acc[kBatch];
-#pragma unroll
-        for (int b = 0; b < kBatch; ++b) acc[b] = 0.f;
-        float s_prev = 0.f;
+        float s0 = 0.f, s1 = 0.f;  // scales of the (at most kLag = 2) groups awaiting read-back
+        static_assert(kLag == 2, "the read-back queue below holds two groups");
 
-        // fold group j's result (tensor-memory buffer j % kDBuffers) into acc
-        auto readback = [&](int j, float sg) {
-            const int db = j % kDBuffers;
-            ok = __all_sync(0xffffffffu, mbar_wait_bounded(d_full + 8 * db, (j / kDBuffers) & 1) && ok);
+        auto readback = [&](int jr, float sg) {
+            const int db = jr % kDBuf;
+            ok = ok && __all_sync(0xffffffffu, mbar_wait_bounded(done + 8 * db, (jr / kDBuf) & 1));
+            if (!ok) return;
             tc_fence_after();
             uint32_t v[kBatch];
-            tmem_ld16(tmem_d + db * kBatch + lane_off, v);
-            tc_fence_before();
-            mbar_arrive(d_free + 8 * db);
+            tmem_ld16(tt + kDCol0 + db * kBatch, v);
 #pragma unroll
             for (int b = 0; b < kBatch; ++b) acc[b] = fmaf(sg, __uint_as_float(v[b]), acc[b]);
         };
 
-        for (int j = 0; j < G && ok; ++j) {
-            const int s = j / kStageGroups, gi = j % kStageGroups, slot = s % kStages;
-            const int ab = j % kABuffers;
-            const float sg = bf16_bits_to_f32(__ldg(srow + j));
-            if (gi == 0) ok = __all_sync(0xffffffffu, mbar_wait_bounded(stage_full + 8 * slot, (s / kStages) & 1));
-            if (!ok) break;
-            uint32_t w[12];
-            const uint4 *src = reinterpret_cast<const uint4 *>(smem + SmemLayout::packed_off + slot * kPackedBytes +
-                                                               r * kPitch * 4 + gi * kBytesPerGroup);
+        Walk walk(p);
+        int64_t t;
+        int g0, len, stage = 0, j = 0, seg = 0;
+        while (ok && walk.next(t, g0, len)) {
 #pragma unroll
-            for (int i = 0; i < 3; ++i) {
-                const uint4 q = src[i];
-                w[4 * i] = q.x;
-                w[4 * i + 1] = q.y;
-                w[4 * i + 2] = q.z;
-                w[4 * i + 3] = q.w;
+            for (int b = 0; b < kBatch; ++b) acc[b] = 0.f;
+            int pend = 0;
+            const int64_t n = t * kRows + r;
+            for (int gs = 0; gs < len && ok; gs += kStageGroups) {
+                const int ns = min(kStageGroups, len - gs);
+                const int slot = stage % kStages;
+                ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar_full + 8 * slot, (stage / kStages) & 1));
+                if (!ok) break;
+                const uint8_t *pk = smem + SmemLayout::stage_off + slot * kStageBytes + kXBytes;
+                const uint16_t *sc = reinterpret_cast<const uint16_t *>(smem + SmemLayout::scale_off +
+                                                                        slot * kScaleSlotBytes) + r;
+                const bool box3 = ns == kStageGroups && p.has_w3;
+                for (int jj = 0; jj < ns; ++jj, ++j) {
+                    const float sg = bf16_bits_to_f32(sc[jj * kRows]);
+                    const uint4 *src = reinterpret_cast<const uint4 *>(
+                        box3 ? pk + r * (kPitch3 * 4) + jj * kBytesPerGroup : pk + jj * kBox1Bytes + r * kBytesPerGroup);
+                    uint32_t w[kWordsPerGroup];
+#pragma unroll
+                    for (int i = 0; i < 3; ++i) {
+                        const uint4 q = src[i];
+                        w[4 * i] = q.x;
+                        w[4 * i + 1] = q.y;
+                        w[4 * i + 2] = q.z;
+                        w[4 * i + 3] = q.w;
+                    }
+                    if (jj == ns - 1) mbar_arrive(bar_empty + 8 * slot);
+                    uint32_t a[64];
+                    group_levels(w, a);
+                    const int ab = j % kABuf;
+                    if (j >= kABuf) {  // the MMAs of group j - kABuf have read this A buffer
+                        const int jp = j - kABuf;
+                        ok = __all_sync(0xffffffffu, mbar_wait_bounded(done + 8 * (jp % kDBuf), (jp / kDBuf) & 1));
+                        if (!ok) break;
+                    }
+                    tc_fence_after();
+                    tmem_st64(tt + ab * kACols, a);
+                    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+                    tc_fence_before();
+                    mbar_arrive(afull + 8 * ab);
+                    if (pend == 2) {
+                        readback(j - 2, s0);
+                        s0 = s1;
+                        pend = 1;
+                    }
+                    if (pend == 0) s0 = sg;
+                    else s1 = sg;
+                    ++pend;
+                }
+                ++stage;
             }
-            if (gi == kStageGroups - 1 || j == G - 1) mbar_arrive(stage_empty + 8 * slot);
-            uint32_t out[64];
-            expand_levels<0>(w, out);
-            ok = __all_sync(0xffffffffu, mbar_wait_bounded(a_free + 8 * ab, ((j / kABuffers) & 1) ^ 1));
-            if (!ok) break;
-            tc_fence_after();
-            tmem_st64(tmem_a + ab * kAColsPerGroup + lane_off, out);
-            asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-            tc_fence_before();
-            mbar_arrive(a_full + 8 * ab);
-            if (j > 0) readback(j - 1, s_prev);
-            s_prev = sg;
-        }
-        if (ok && G > 0) readback(G - 1, s_prev);
-        if (ok && n < p.N) {
+            if (pend >= 1) readback(j - pend, s0);
+            if (pend == 2) readback(j - 1, s1);
+            if (len == p.G) {  // the whole tile is this CTA's: store y
+                if (n < p.N) {
 #pragma unroll
-            for (int b = 0; b < kBatch; ++b)
-                if (b < p.M) p.y[static_cast<int64_t>(b) * p.N + n] = f32_to_bf16_rn(acc[b]);
+                    for (int b = 0; b < kBatch; ++b)
+                        if (b < p.M) p.y[static_cast<int64_t>(b) * p.N + n] = f32_to_bf16_rn(acc[b]);
+                }
+            } else {  // shared tile: fp32 partial sums for the fix-up kernel
+                float *dst = p.partial + (static_cast<int64_t>(blockIdx.x) * 2 + (seg == 0 ? 0 : 1)) * kBatch * kRows + r;
+#pragma unroll
+                for (int b = 0; b < kBatch; ++b)
+                    if (b < p.M) dst[b * kRows] = acc[b];
+            }
+            ++seg;
         }
     }
 
@@ -285,6 +510,68 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(const __grid_con
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
     }
+}
+
+// Tiles shared by several CTAs: block i-1 handles the tile that unit_begin(i)
+// falls inside (when it is the first such boundary of that tile) and adds the
+// partial sums of the CTAs that cover it, in CTA order.
+__global__ void __launch_bounds__(kRows) decode_tc_fixup_kernel(const __grid_constant__ FixupParams p) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const int i = blockIdx.x + 1;
+    const int64_t u = unit_begin(i, p.U, p.P);
+    const int64_t t = u / p.G;
+    const int64_t t0 = t * p.G, t1 = t0 + p.G;
+    if (u == t0 || unit_begin(i - 1, p.U, p.P) > t0) return;
+    const int r = threadIdx.x;
+    const int64_t n = t * kRows + r;
+    if (n >= p.N) return;
+    float acc[kBatch];
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) acc[b] = 0.f;
+    // contributors in rounds of 4 whose loads are all issued before the adds
+    constexpr int kRound = 4;
+    for (int c = i - 1; c < p.P;) {
+        const float *src[kRound];
+        int cnt = 0;
+        for (; cnt < kRound && c < p.P; ++c) {
+            const int64_t uc = unit_begin(c, p.U, p.P);
+            if (uc >= t1) break;
+            const int slot = (uc / p.G == t) ? 0 : 1;
+            src[cnt++] = p.partial + (static_cast<int64_t>(c) * 2 + slot) * kBatch * kRows + r;
+        }
+        float v[kRound][kBatch];
+#pragma unroll
+        for (int q = 0; q < kRound; ++q)
+#pragma unroll
+            for (int b = 0; b < kBatch; ++b) v[q][b] = (q < cnt && b < p.M) ? __ldcg(src[q] + b * kRows) : 0.f;
+#pragma unroll
+        for (int q = 0; q < kRound; ++q)
+#pragma unroll
+            for (int b = 0; b < kBatch; ++b)
+                if (q < cnt) acc[b] += v[q][b];
+        if (cnt < kRound) break;
+    }
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b)
+        if (b < p.M) p.y[static_cast<int64_t>(b) * p.N + n] = f32_to_bf16_rn(acc[b]);
+}
+
+struct LaunchPlan {
+    int P;              // CTAs (one per SM at most)
+    int64_t U;          // units
+    int64_t ws_floats;  // partial-sum workspace (0 when one CTA does everything)
+};
+
+inline LaunchPlan plan(int64_t N, int64_t K, int num_sms) {
+    LaunchPlan L;
+    const int64_t T = (N + kRows - 1) / kRows;
+    L.U = T * (K / kGroup);
+    int64_t P = L.U / kMinUnitsPerCta;
+    if (P > num_sms) P = num_sms;
+    if (P < 1) P = 1;
+    L.P = static_cast<int>(P);
+    L.ws_floats = L.P > 1 ? static_cast<int64_t>(L.P) * 2 * kBatch * kRows : 0;
+    return L;
 }
 
 }  // namespace decode_tc

@@ -83,19 +83,32 @@ __host__ __device__ constexpr uint32_t make_idesc(int m, int n) {
            | (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(m >> 4) << 24);
 }
 
+// The descriptor of the same tile `bytes` further on (the start address field
+// counts 16-byte units and never carries out for shared-memory addresses).
+__device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t bytes) { return desc + (bytes >> 4); }
+
+// tcgen05.mma and tcgen05.commit are single-thread instructions.  These
+// wrappers are called by every lane of a converged warp and issue from one
+// lane chosen by elect.sync: with warp-uniform operands the issuing loop costs
+// a few instructions per MMA (issued from one thread inside a branch it costs
+// several times more and, at small N, limits the tensor pipe).
 __device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                           uint32_t accumulate) {
     asm volatile(
-        "{\n\t.reg .pred p;\n\t"
+        "{\n\t.reg .pred p, e;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-                 : "memory");
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(bar)
+        : "memory");
 }
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -205,28 +218,28 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             }
         }
     } else if (warp == 1) {
-        // ---- MMA issuer ----
-        if (lane == 0) {
-            for (int s = 0; s < nstages && ok; ++s) {
-                const int slot = s % kStages;
-                const uint32_t par = static_cast<uint32_t>(s / kStages) & 1u;
-                ok = mbar_wait_bounded(bar_full_a + 8 * slot, par) && mbar_wait_bounded(bar_full_b + 8 * slot, par);
-                if (!ok) break;
-                tc_fence_after();
-                const uint32_t a0 = a_base + slot * 2 * kABytes;
-                const uint32_t b0 = b_base + slot * kBBytes;
+        // ---- MMA issuer: the whole warp runs the loop, one elected lane issues ----
+        const uint64_t adesc0 = sw128_kmajor_desc(a_base), bdesc0 = sw128_kmajor_desc(b_base);
+        const uint32_t d1 = tmem + static_cast<uint32_t>(p.tile_n);
+        for (int s = 0; s < nstages && ok; ++s) {
+            const int slot = s % kStages;
+            const uint32_t par = static_cast<uint32_t>(s / kStages) & 1u;
+            ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar_full_a + 8 * slot, par) &&
+                                             mbar_wait_bounded(bar_full_b + 8 * slot, par));
+            if (!ok) break;
+            tc_fence_after();
+            const uint64_t ad = desc_add(adesc0, slot * 2 * kABytes);
+            const uint64_t bd0 = desc_add(bdesc0, slot * kBBytes);
 #pragma unroll
-                for (int kk = 0; kk < kStageK / 16; ++kk) {
-                    const uint64_t bd = sw128_kmajor_desc(b0 + kk * 32);
-                    const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
-                    umma_bf16(tmem, sw128_kmajor_desc(a0 + kk * 32), bd, p.idesc, acc);
-                    umma_bf16(tmem + static_cast<uint32_t>(p.tile_n), sw128_kmajor_desc(a0 + kABytes + kk * 32), bd,
-                              p.idesc, acc);
-                }
-                umma_commit(bar_empty + 8 * slot);  // frees the stage once these MMAs have read it
+            for (int kk = 0; kk < kStageK / 16; ++kk) {
+                const uint64_t bd = desc_add(bd0, kk * 32);
+                const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
+                umma_bf16(tmem, desc_add(ad, kk * 32), bd, p.idesc, acc);
+                umma_bf16(d1, desc_add(ad, kABytes + kk * 32), bd, p.idesc, acc);
             }
-            umma_commit(bar_acc);  // all accumulation done
+            umma_commit(bar_empty + 8 * slot);  // frees the stage once these MMAs have read it
         }
+        if (ok) umma_commit(bar_acc);  // all accumulation done
     } else {
         // ---- B producers: dequantize one W row per thread ----
         const int t = threadIdx.x - 64;  // 0..255
