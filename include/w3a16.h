@@ -120,6 +120,24 @@ w3_status w3a16_gemm(const uint16_t *x, const int32_t *packed, const uint16_t *s
                      int64_t M, int64_t N, int64_t K, w3_stream_t stream);
 
 /*
+ * w3a16_gemm_noalloc -- the same product y = x * W^T as w3a16_gemm, with the
+ * same arguments, checks, errors and results, that allocates nothing: the
+ * tensor-core decode (5 <= M <= 16, N >= 256) keeps its fp32 partial sums in a
+ * fixed scratch array inside the library (about 5 MB of device memory per
+ * device, sized for up to 160 SMs) instead of a stream-ordered allocation;
+ * every other shape runs exactly as in w3a16_gemm.  The format paper has no
+ * counterpart to this call; it is for callers that may not allocate.
+ *   - W3_ERR_UNSUPPORTED if the decode would need more scratch than the array
+ *     holds (a GPU with more than 160 SMs).
+ *   - The scratch is shared by all calls on a device: calls that overlap in
+ *     time (on different streams, or from different host threads) race on it
+ *     and may return wrong results.  Calls on one stream are ordered and safe.
+ *   - The scratch needs no initialisation: each call writes every slot it reads.
+ */
+w3_status w3a16_gemm_noalloc(const uint16_t *x, const int32_t *packed, const uint16_t *scales, uint16_t *y,
+                             int64_t M, int64_t N, int64_t K, w3_stream_t stream);
+
+/*
  * w3_check_device_error -- synchronise `stream`, then report and clear the
  * current device's error flag: W3_OK, or W3_ERR_TIMEOUT if a kernel of this
  * library gave up a bounded wait since the last check.  W3_ERR_CUDA if the

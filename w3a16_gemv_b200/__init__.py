@@ -19,6 +19,7 @@ from ._binding import (  # noqa: F401
     w3_packed_words_per_row,
     w3_unpack,
     w3a16_gemm,
+    w3a16_gemm_noalloc,
 )
 
 __all__ = [
@@ -32,4 +33,5 @@ __all__ = [
     "w3_packed_words_per_row",
     "w3_unpack",
     "w3a16_gemm",
+    "w3a16_gemm_noalloc",
 ]

@@ -41,6 +41,7 @@ SIGNATURES = [
     ("w3_unpack", ctypes.c_int, [_P, _P, _I64, _I64, _P]),
     ("w3_dequant_f32", ctypes.c_int, [_P, _P, _P, _I64, _I64, _P]),
     ("w3a16_gemm", ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P]),
+    ("w3a16_gemm_noalloc", ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P]),
     ("w3_check_device_error", ctypes.c_int, [_P]),
 ]
 
@@ -152,6 +153,17 @@ def w3_dequant_f32(packed: torch.Tensor, scales: torch.Tensor, K: int, out: torc
 def w3a16_gemm(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, out: torch.Tensor | None = None,
                stream=None) -> torch.Tensor:
     """y = x W^T, x bf16 [M,K], packed int32 [N,3K/32], scales bf16 [N,K/128] -> y bf16 [M,N]."""
+    return _gemm("w3a16_gemm", x, packed, scales, out, stream)
+
+
+def w3a16_gemm_noalloc(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
+                       out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """w3a16_gemm with the library's fixed scratch instead of an allocation (overlapping calls race)."""
+    return _gemm("w3a16_gemm_noalloc", x, packed, scales, out, stream)
+
+
+def _gemm(entry: str, x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, out: torch.Tensor | None,
+          stream) -> torch.Tensor:
     _need(x, torch.bfloat16, "x")
     _need(packed, torch.int32, "packed")
     _need(scales, torch.bfloat16, "scales")
@@ -164,8 +176,8 @@ def w3a16_gemm(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, out:
     _need(out, torch.bfloat16, "out")
     if tuple(out.shape) != (M, N):
         raise ValueError("out must be [M, N]")
-    _check(lib().w3a16_gemm(x.data_ptr(), packed.data_ptr(), scales.data_ptr(), out.data_ptr(), M, N, K,
-                            _stream(stream)), "w3a16_gemm")
+    _check(getattr(lib(), entry)(x.data_ptr(), packed.data_ptr(), scales.data_ptr(), out.data_ptr(), M, N, K,
+                                 _stream(stream)), entry)
     return out
 
 

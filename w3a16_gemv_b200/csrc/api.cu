@@ -349,6 +349,33 @@ w3_status launch_decode(const uint16_t *x, const int32_t *packed, const uint16_t
     return e == cudaSuccess ? W3_OK : W3_ERR_CUDA;
 }
 
+// Fixed scratch of w3a16_gemm_noalloc: the fp32 partial sums of the tensor-core
+// decode for up to kNoAllocMaxCtas CTAs (one per SM).  Every slot the fix-up
+// kernel reads is written by the main kernel of the same call, so nothing in
+// it has to start at zero.
+constexpr int kNoAllocMaxCtas = 160;
+constexpr int64_t kNoAllocScratchFloats = int64_t(kNoAllocMaxCtas) * 2 * decode_tc::kBatch * decode_tc::kRows;
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchFloats];
+
+struct NoAllocState {
+    std::once_flag once;
+    float *scratch = nullptr;
+};
+NoAllocState g_noalloc[kMaxDevices];
+
+// Address of the scratch on the current device (looked up once per device, with
+// that device current).
+float *noalloc_scratch() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    NoAllocState &st = g_noalloc[dev];
+    std::call_once(st.once, [&] {
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) == cudaSuccess) st.scratch = static_cast<float *>(ptr);
+    });
+    return st.scratch;
+}
+
 }  // namespace
 }  // namespace w3
 
@@ -464,6 +491,29 @@ w3_status w3a16_gemm(const uint16_t *x, const int32_t *packed, const uint16_t *s
     }
     if (partial && cudaFreeAsync(partial, st) != cudaSuccess && status == W3_OK) status = W3_ERR_CUDA;
     return status;
+}
+
+w3_status w3a16_gemm_noalloc(const uint16_t *x, const int32_t *packed, const uint16_t *scales, uint16_t *y,
+                             int64_t M, int64_t N, int64_t K, w3_stream_t stream) {
+    if (!x || !packed || !scales || !y) return W3_ERR_NULL;
+    if (w3_status s = check_nk(N, K)) return s;
+    if (M < 1 || M > kMaxDim || M * K > kMaxElems || M * N > kMaxElems) return W3_ERR_SHAPE;
+    if (!aligned16(x) || !aligned16(packed) || !aligned16(scales) || !aligned16(y)) return W3_ERR_ALIGN;
+    const int64_t ybytes = M * N * 2;
+    if (overlaps(y, ybytes, x, M * K * 2) || overlaps(y, ybytes, packed, N * K * 3 / 8) ||
+        overlaps(y, ybytes, scales, N * (K / kGroup) * 2))
+        return W3_ERR_ALIAS;
+    int sms;
+    if (w3_status s = device_setup(&sms)) return s;
+    // Only the tensor-core decode (W3_DECODE_TC_MIN_M <= M <= 16, N >= 256) uses
+    // scratch; every other shape takes w3a16_gemm's path, which allocates nothing.
+    if (M > 16 || M < W3_DECODE_TC_MIN_M || N < decode_tc::kRows) return w3a16_gemm(x, packed, scales, y, M, N, K, stream);
+    const decode_tc::LaunchPlan tplan = decode_tc::plan(N, K, sms);
+    if (tplan.ws_floats > kNoAllocScratchFloats) return W3_ERR_UNSUPPORTED;
+    float *scratch = noalloc_scratch();
+    if (!scratch) return W3_ERR_CUDA;
+    return launch_decode_tc(x, packed, scales, y, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K),
+                            tplan, scratch, reinterpret_cast<cudaStream_t>(stream));
 }
 
 w3_status w3_check_device_error(w3_stream_t stream) {
