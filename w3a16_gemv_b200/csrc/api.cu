@@ -353,7 +353,7 @@ w3_status launch_decode(const uint16_t *x, const int32_t *packed, const uint16_t
 // decode for up to kNoAllocMaxCtas CTAs (one per SM).  Every slot the fix-up
 // kernel reads is written by the main kernel of the same call, so nothing in
 // it has to start at zero.
-constexpr int kNoAllocMaxCtas = 160;
+constexpr int kNoAllocMaxCtas = 160 * decode_tc::kCtasPerSm;
 constexpr int64_t kNoAllocScratchFloats = int64_t(kNoAllocMaxCtas) * 2 * decode_tc::kBatch * decode_tc::kRows;
 static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchFloats];
 

@@ -27,15 +27,15 @@
 //    pair schedule as the mma.sync decode: each LOP3 drops two codes into the
 //    mantissa of bf16 128.0 at bit offsets e_lo, e_hi, the exact value
 //    128 + c*2^e -- and one bf16x2 FMA per pair, v*2^-e - (128*2^-e + 4),
-//    turns each into the exact level q = c - 4.  The 64 words of a group go
-//    to the thread's tensor-memory lane with one tcgen05.st: the A operand,
-//    three group buffers per tile.
+//    turns each into the exact level q = c - 4 (the ten FMA constants are
+//    pinned in registers).  The group's 64 words go to the thread's
+//    tensor-memory lane (two tcgen05.st): the A operand.
 //  * One thread issues 8 tcgen05.mma per group and tile (A from tensor memory,
 //    B = permuted x from shared memory) into a fresh per-group fp32
 //    accumulator of 16 columns (four buffers per tile).
 //  * The row threads read each group's 16 results back two groups later
 //    (tcgen05.ld) and add s[n,g] * D to fp32 registers: the group scale is
-//    applied in fp32 and nothing is rounded before the final bf16 store.
+//    applied in fp32 and nothing is rounded before the bf16 store.
 #pragma once
 
 #include "common.cuh"
@@ -59,7 +59,15 @@ constexpr int kTiles = 2;                         // row tiles per CTA, sharing 
 constexpr int kRows = kTiles * kTileRows;         // 256 rows per CTA (one TMA box)
 constexpr int kBatch = 16;                        // UMMA N
 constexpr int kStageGroups = 3;
-constexpr int kStages = 4;
+// Resident CTAs per SM and, with them, the per-CTA budgets of shared and
+// tensor memory: one CTA with 4 stages and 3 A buffers per tile, or two CTAs
+// with 2 stages and 1 A buffer per tile each (twice the row warps per SM).
+#ifndef W3_DECODE_TC_CTAS_PER_SM
+#define W3_DECODE_TC_CTAS_PER_SM 1
+#endif
+constexpr int kCtasPerSm = W3_DECODE_TC_CTAS_PER_SM;
+static_assert(kCtasPerSm == 1 || kCtasPerSm == 2, "one or two CTAs per SM");
+constexpr int kStages = kCtasPerSm == 1 ? 4 : 2;
 constexpr int kPitch3 = kStageGroups * kWordsPerGroup;        // 36 words: rows of a 3-group box
 constexpr int kPitch1 = kWordsPerGroup;                       // 12 words: rows of a 1-group box
 constexpr int kBox1Bytes = kRows * kPitch1 * 4;               // 12 KB
@@ -67,17 +75,19 @@ constexpr int kXBox = kBatch * 64 * 2;                        // 2 KB: [16 rows]
 constexpr int kXGroupBytes = 2 * kXBox;                       // 4 KB
 constexpr int kXBytes = kStageGroups * kXGroupBytes;          // 12 KB
 constexpr int kStageBytes = kXBytes + kStageGroups * kBox1Bytes;  // 48 KB
-constexpr int kABuf = 3;                                      // A buffers (one group each) per tile
+constexpr int kABuf = kCtasPerSm == 1 ? 3 : 1;                // A buffers (one group each) per tile
 constexpr int kDBuf = 4;                                      // accumulators per tile
 constexpr int kLag = 2;                                       // groups between MMA and read-back
 constexpr int kACols = 64;                                    // 128 codes, two bf16 per column
 constexpr int kDCol0 = kABuf * kACols;                        // 192
 constexpr int kTileCols = kDCol0 + kDBuf * kBatch;            // 256 columns per tile
-constexpr int kTmemCols = kTiles * kTileCols;                 // 512: one CTA per SM
+constexpr int kTmemCols = kTiles * kTileCols;                 // 512 or 256 (two CTAs per SM)
+static_assert(kTmemCols * kCtasPerSm <= 512, "tensor memory per SM");
 constexpr int kRowWarps = kTiles * 4;
 constexpr int kScaleWarp = 2 + kRowWarps;                     // warp 10
 constexpr int kThreads = (3 + kRowWarps) * 32;                // load, MMA, row warps, scale warp
 constexpr int kScaleSlotBytes = kStageGroups * kRows * 2;     // [3 groups][256 rows] bf16
+
 #ifndef W3_DECODE_TC_MIN_UNITS
 #define W3_DECODE_TC_MIN_UNITS 6
 #endif
@@ -95,8 +105,8 @@ struct SmemLayout {
     static constexpr int stage_off = 0;  // [kStages]{x: [3][2 boxes], packed}
     static constexpr int scale_off = stage_off + kStages * kStageBytes;  // [kStages][3][256] bf16
     static constexpr int bar_off = scale_off + kStages * kScaleSlotBytes;
-    // full, empty, bready [kStages]; a_full [kTiles][kABuf]; done [kTiles][kDBuf] (the MMAs of a group)
-    static constexpr int nbars = 3 * kStages + kTiles * kABuf + kTiles * kDBuf;
+    // full, empty, bready [kStages]; a_full [kTiles][kABuf]; done [kDBuf] (the MMAs of a group, both tiles)
+    static constexpr int nbars = 3 * kStages + kTiles * kABuf + kDBuf;
     static constexpr int tmem_slot_off = bar_off + nbars * 8;
     static constexpr int total = tmem_slot_off + 16 + 1024;  // + slack for 1024-byte alignment
 };
@@ -129,22 +139,57 @@ __host__ __device__ inline int64_t unit_begin(int c, int64_t U, int P) { return 
 
 // ---- compile-time constants of the pair schedule ----------------------------------
 
+// bf16x2 (2^-e_lo, 2^-e_hi) for pair i: the scaling of x' in the pair's two slots.
+__host__ __device__ constexpr uint32_t pair_mul(int i) {
+    return static_cast<uint32_t>((127 - pair_spec(i).elo) << 7) | (static_cast<uint32_t>(127 - pair_spec(i).ehi) << 23);
+}
 // bf16 bits of a positive integer v < 256 with at most 8 significant bits.
 __host__ __device__ constexpr uint32_t bf16_of_int(int v) {
     int e = 0;
     while ((v >> (e + 1)) != 0) ++e;
     return static_cast<uint32_t>(((127 + e) << 7) | (((v - (1 << e)) << 7) >> e));
 }
-// bf16x2 (2^-e_lo, 2^-e_hi) and (-(128*2^-e_lo + 4), -(128*2^-e_hi + 4)) for pair i.
-__host__ __device__ constexpr uint32_t pair_mul(int i) {
-    return static_cast<uint32_t>((127 - pair_spec(i).elo) << 7) | (static_cast<uint32_t>(127 - pair_spec(i).ehi) << 23);
-}
+// bf16x2 (-(128*2^-e_lo + 4), -(128*2^-e_hi + 4)) for pair i.
 __host__ __device__ constexpr uint32_t pair_add(int i) {
     return (0x8000u | bf16_of_int((128 >> pair_spec(i).elo) + 4)) |
            ((0x8000u | bf16_of_int((128 >> pair_spec(i).ehi) + 4)) << 16);
 }
 static_assert(bf16_of_int(132) == 0x4304u && bf16_of_int(12) == 0x4140u && bf16_of_int(68) == 0x4288u,
               "bf16 encoding of the level offsets");
+// The (e_lo, e_hi) combinations of the pair schedule, and the combination of pair i.
+constexpr int kOffsetKinds = 5;
+__host__ __device__ constexpr int offset_kind(int elo, int ehi) {
+    return elo == 4 && ehi == 0 ? 0 : elo == 1 && ehi == 3 ? 1 : elo == 4 && ehi == 3 ? 2 : elo == 1 && ehi == 0 ? 3 : 4;
+}
+__host__ __device__ constexpr int pair_kind(int i) { return offset_kind(pair_spec(i).elo, pair_spec(i).ehi); }
+__host__ __device__ constexpr bool pair_kinds_complete() {
+    for (int i = 0; i < 16; ++i) {
+        const int k = pair_kind(i);
+        const int elo = k == 0 ? 4 : k == 1 ? 1 : k == 2 ? 4 : k == 3 ? 1 : 2;
+        const int ehi = k == 0 ? 0 : k == 1 ? 3 : k == 2 ? 3 : k == 3 ? 0 : 1;
+        if (elo != pair_spec(i).elo || ehi != pair_spec(i).ehi) return false;
+    }
+    return true;
+}
+static_assert(pair_kinds_complete(), "every pair's offsets are one of the five kinds");
+
+// The FMA constants of the five kinds, held in registers.  Written through
+// opaque moves so that the compiler keeps them instead of re-creating them
+// before every use.
+struct LevelConsts {
+    uint32_t mul[kOffsetKinds], add[kOffsetKinds];
+    __device__ __forceinline__ LevelConsts() {
+#pragma unroll
+        for (int k = 0; k < kOffsetKinds; ++k) {
+            const int elo = k == 0 ? 4 : k == 1 ? 1 : k == 2 ? 4 : k == 3 ? 1 : 2;
+            const int ehi = k == 0 ? 0 : k == 1 ? 3 : k == 2 ? 3 : k == 3 ? 0 : 1;
+            const uint32_t m = static_cast<uint32_t>((127 - elo) << 7) | (static_cast<uint32_t>(127 - ehi) << 23);
+            const uint32_t a = (0x8000u | bf16_of_int((128 >> elo) + 4)) | ((0x8000u | bf16_of_int((128 >> ehi) + 4)) << 16);
+            asm volatile("mov.b32 %0, %1;" : "=r"(mul[k]) : "r"(m));
+            asm volatile("mov.b32 %0, %1;" : "=r"(add[k]) : "r"(a));
+        }
+    }
+};
 // __byte_perm selector taking element lo of word a and element hi of word b.
 __host__ __device__ constexpr uint32_t pair_sel(int i) {
     const uint32_t b0 = 2u * (pair_spec(i).lo & 1), b2 = 4u + 2u * (pair_spec(i).hi & 1);
@@ -169,20 +214,15 @@ __device__ __forceinline__ void umma_ts(uint32_t tmem_d, uint32_t tmem_a, uint64
         : "memory");
 }
 
-// 64 consecutive 32-bit columns of this thread's TMEM lane from registers.
-__device__ __forceinline__ void tmem_st64(uint32_t taddr, const uint32_t (&v)[64]) {
+// 32 consecutive 32-bit columns of this thread's TMEM lane from registers.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
     asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x64.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,"
-        "%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,%64};" ::"r"(taddr),
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
         "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
         "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]),
         "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]),
-        "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31]), "r"(v[32]), "r"(v[33]), "r"(v[34]), "r"(v[35]),
-        "r"(v[36]), "r"(v[37]), "r"(v[38]), "r"(v[39]), "r"(v[40]), "r"(v[41]), "r"(v[42]), "r"(v[43]), "r"(v[44]),
-        "r"(v[45]), "r"(v[46]), "r"(v[47]), "r"(v[48]), "r"(v[49]), "r"(v[50]), "r"(v[51]), "r"(v[52]), "r"(v[53]),
-        "r"(v[54]), "r"(v[55]), "r"(v[56]), "r"(v[57]), "r"(v[58]), "r"(v[59]), "r"(v[60]), "r"(v[61]), "r"(v[62]),
-        "r"(v[63])
+        "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
         : "memory");
 }
 
@@ -196,15 +236,19 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-// A group's 128 codes (12 words) as 64 bf16x2 words of exact levels, in pair order:
-// word 16*b + i holds codes (lo_i, hi_i) of block b.
-__device__ __forceinline__ void group_levels(const uint32_t (&w)[kWordsPerGroup], uint32_t (&a)[64]) {
+// Half H of a group's 128 codes (blocks 2H, 2H+1; 6 of the 12 words) as 32
+// bf16x2 words of exact levels in pair order: word 16*b + i holds codes
+// (lo_i, hi_i) of block 2H + b.
+template <int H>
+__device__ __forceinline__ void half_levels(const uint32_t (&w)[kWordsPerGroup], const LevelConsts &lc,
+                                            uint32_t (&a)[32]) {
 #pragma unroll
-    for (int b = 0; b < 4; ++b) {
+    for (int b = 0; b < 2; ++b) {
+        const int bb = 2 * H + b;
         uint32_t blk[16];
-        decode::unpack_block(w[3 * b], w[3 * b + 1], w[3 * b + 2], blk);
+        decode::unpack_block(w[3 * bb], w[3 * bb + 1], w[3 * bb + 2], blk);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) a[16 * b + i] = bf16x2_fma(blk[i], pair_mul(i), pair_add(i));
+        for (int i = 0; i < 16; ++i) a[16 * b + i] = bf16x2_fma(blk[i], lc.mul[pair_kind(i)], lc.add[pair_kind(i)]);
     }
 }
 
@@ -260,14 +304,15 @@ struct Walk {
     }
 };
 
-__global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_constant__ Params p) {
+__global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_tc_kernel(const __grid_constant__ Params p) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // 1024-byte aligned, derived from the __shared__ array so that accesses stay shared-memory ones
+    uint8_t *smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
     const uint32_t sbase = smem_addr(smem);
     const uint32_t bars = sbase + SmemLayout::bar_off;
     const uint32_t bar_full = bars, bar_empty = bars + 8 * kStages, bar_bready = bars + 16 * kStages;
     const uint32_t bar_afull = bars + 24 * kStages;                // [kTiles][kABuf]
-    const uint32_t bar_done = bar_afull + 8 * kTiles * kABuf;      // [kTiles][kDBuf]
+    const uint32_t bar_done = bar_afull + 8 * kTiles * kABuf;      // [kDBuf]
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + SmemLayout::tmem_slot_off);
 
     const int warp = threadIdx.x >> 5;
@@ -283,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
             mbar_init(bar_bready + 8 * s, 1);
         }
         for (int b = 0; b < kTiles * kABuf; ++b) mbar_init(bar_afull + 8 * b, kTileRows);
-        for (int b = 0; b < kTiles * kDBuf; ++b) mbar_init(bar_done + 8 * b, 1);
+        for (int b = 0; b < kDBuf; ++b) mbar_init(bar_done + 8 * b, 1);
         mbar_init_fence();
     }
     if (warp == 1) {
@@ -373,8 +418,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
                             if (kk == 0) umma_ts<false>(dcol, acol, bd, p.idesc);
                             else umma_ts<true>(dcol, acol + kk * 8, bd, p.idesc);
                         }
-                        umma_commit(bar_done + 8 * (tile * kDBuf + db));  // A read, D written
                     }
+                    if (!ok) break;
+                    umma_commit(bar_done + 8 * db);  // both tiles: A read, D written
                 }
                 if (!ok) break;
                 umma_commit(bar_empty + 8 * slot);
@@ -415,11 +461,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         const int quarter = warp & 3;  // a warp reaches TMEM lanes 32*(warp % 4) .. +31
         const int r = tile * kTileRows + quarter * 32 + lane;
         const uint32_t tt = tmem + tile * kTileCols + (static_cast<uint32_t>(quarter * 32) << 16);
-        const uint32_t afull = bar_afull + 8 * tile * kABuf, done = bar_done + 8 * tile * kDBuf;
+        const uint32_t afull = bar_afull + 8 * tile * kABuf, done = bar_done;
         float acc[kBatch];
         float s0 = 0.f, s1 = 0.f;  // scales of the (at most kLag = 2) groups awaiting read-back
         static_assert(kLag == 2, "the read-back queue below holds two groups");
 
+        const LevelConsts lc;
         auto readback = [&](int jr, float sg) {
             const int db = jr % kDBuf;
             ok = ok && __all_sync(0xffffffffu, mbar_wait_bounded(done + 8 * db, (jr / kDBuf) & 1));
@@ -462,8 +509,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
                         w[4 * i + 3] = q.w;
                     }
                     if (jj == ns - 1) mbar_arrive(bar_empty + 8 * slot);
-                    uint32_t a[64];
-                    group_levels(w, a);
+                    // the group's levels, one half (blocks 0-1, then 2-3) at a time
+                    uint32_t a[32];
+                    half_levels<0>(w, lc, a);
                     const int ab = j % kABuf;
                     if (j >= kABuf) {  // the MMAs of group j - kABuf have read this A buffer
                         const int jp = j - kABuf;
@@ -471,7 +519,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
                         if (!ok) break;
                     }
                     tc_fence_after();
-                    tmem_st64(tt + ab * kACols, a);
+                    tmem_st32(tt + ab * kACols, a);
+                    half_levels<1>(w, lc, a);
+                    tmem_st32(tt + ab * kACols + 32, a);
                     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
                     tc_fence_before();
                     mbar_arrive(afull + 8 * ab);
@@ -567,7 +617,7 @@ inline LaunchPlan plan(int64_t N, int64_t K, int num_sms) {
     const int64_t T = (N + kRows - 1) / kRows;
     L.U = T * (K / kGroup);
     int64_t P = L.U / kMinUnitsPerCta;
-    if (P > num_sms) P = num_sms;
+    if (P > static_cast<int64_t>(num_sms) * kCtasPerSm) P = static_cast<int64_t>(num_sms) * kCtasPerSm;
     if (P < 1) P = 1;
     L.P = static_cast<int>(P);
     L.ws_floats = L.P > 1 ? static_cast<int64_t>(L.P) * 2 * kBatch * kRows : 0;
