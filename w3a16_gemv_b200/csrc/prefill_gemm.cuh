@@ -13,7 +13,8 @@
 //  * A (x): one tiled TMA copy per 128-row tile and stage, 128-byte swizzle,
 //    the canonical K-major layout the UMMA descriptors describe.
 //  * B (W): 8 dequantizing warps, one W row per thread.  A stage of a row is
-//    64 codes = 6 packed words (loaded one stage ahead).  Codes are expanded
+//    64 codes = 6 packed words, loaded kPrefetch stages ahead into a register
+//    ring so that the global-load latency hides behind the expansions.  Codes are expanded
 //    in natural k order four at a time: the 12 bits of two code pairs times
 //    0x2001 place each pair's second code 13 bits above its first, so one
 //    LOP3 (mask | bf16 128.0) per pair gives (128 + c_k, 128 + c_k+1) exactly;
@@ -44,6 +45,10 @@ constexpr int kTmemCols = 512;
 constexpr int kABytes = kUmmaM * kStageK * 2;     // 16 KB per 128-row tile and stage
 constexpr int kBBytes = kMaxTileN * kStageK * 2;  // 32 KB per stage (BN rows used)
 constexpr int kStageWords = kStageK * 3 / 32;     // 6 packed words per row and stage
+#ifndef W3_PREFILL_PREFETCH
+#define W3_PREFILL_PREFETCH 4
+#endif
+constexpr int kPrefetch = W3_PREFILL_PREFETCH;      // stages of packed words in flight per thread
 
 struct SmemLayout {
     // all operand buffers are 1024-byte aligned (the 128-byte swizzle period)
@@ -163,7 +168,8 @@ __device__ __forceinline__ void expand_quads(const uint32_t (&w)[kStageWords], u
 
 __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_constant__ Params p) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // 1024-byte aligned, derived from the __shared__ array so that accesses stay shared-memory ones
+    uint8_t *smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
     const uint32_t sbase = smem_addr(smem);
     const uint32_t a_base = sbase + SmemLayout::a_off;
     const uint32_t b_base = sbase + SmemLayout::b_off;
@@ -247,8 +253,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         const bool row_ok = (t < p.tile_n) && (n < p.N);
         const uint32_t *prow = p.packed + static_cast<int64_t>(row_ok ? n : 0) * W;
         const uint16_t *srow = p.scales + static_cast<int64_t>(row_ok ? n : 0) * G;
-        uint32_t w[kStageWords] = {};
-        uint32_t s_next = 0;
+        // register ring: stage s lives in ring[s % kPrefetch]
+        uint32_t ring[kPrefetch][kStageWords] = {};
+        uint32_t ring_s[kPrefetch] = {};
         auto load = [&](int s, uint32_t (&dst)[kStageWords], uint32_t &sc) {
             if (row_ok && s < nstages) {
                 const uint2 *src = reinterpret_cast<const uint2 *>(prow + s * kStageWords);
@@ -262,36 +269,42 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                 sc = h | (h << 16);
             }
         };
-        load(0, w, s_next);
-        for (int s = 0; s < nstages && ok; ++s) {
-            uint32_t cur[kStageWords];
 #pragma unroll
-            for (int i = 0; i < kStageWords; ++i) cur[i] = w[i];
-            const uint32_t s2 = s_next;
-            load(s + 1, w, s_next);  // prefetch the next stage
-            uint32_t out[32];
-            if (row_ok) {
-                expand_quads<0>(cur, s2, out);
-            } else {
+        for (int u = 0; u < kPrefetch; ++u) load(u, ring[u], ring_s[u]);
+        for (int s0 = 0; s0 < nstages && ok; s0 += kPrefetch) {
 #pragma unroll
-                for (int i = 0; i < 32; ++i) out[i] = 0u;
-            }
-            const int slot = s % kStages;
-            const uint32_t round = static_cast<uint32_t>(s / kStages);
-            ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar_empty + 8 * slot, (round & 1u) ^ 1u));
-            if (!ok) break;
-            if (t < p.tile_n) {
-                const uint32_t row = b_base + slot * kBBytes + t * 128;
+            for (int u = 0; u < kPrefetch; ++u) {
+                const int s = s0 + u;
+                if (s >= nstages || !ok) break;
+                uint32_t cur[kStageWords];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const uint32_t dst = row + ((j ^ (t & 7)) << 4);
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(out[4 * j]),
-                                 "r"(out[4 * j + 1]), "r"(out[4 * j + 2]), "r"(out[4 * j + 3])
-                                 : "memory");
+                for (int i = 0; i < kStageWords; ++i) cur[i] = ring[u][i];
+                const uint32_t s2 = ring_s[u];
+                load(s + kPrefetch, ring[u], ring_s[u]);  // refill this ring slot
+                uint32_t out[32];
+                if (row_ok) {
+                    expand_quads<0>(cur, s2, out);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) out[i] = 0u;
                 }
+                const int slot = s % kStages;
+                const uint32_t round = static_cast<uint32_t>(s / kStages);
+                ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar_empty + 8 * slot, (round & 1u) ^ 1u));
+                if (!ok) break;
+                if (t < p.tile_n) {
+                    const uint32_t row = b_base + slot * kBBytes + t * 128;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const uint32_t dst = row + ((j ^ (t & 7)) << 4);
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(out[4 * j]),
+                                     "r"(out[4 * j + 1]), "r"(out[4 * j + 2]), "r"(out[4 * j + 3])
+                                     : "memory");
+                    }
+                }
+                fence_async_smem();
+                mbar_arrive(bar_full_b + 8 * slot);
             }
-            fence_async_smem();
-            mbar_arrive(bar_full_b + 8 * slot);
         }
 
         // ---- epilogue: TMEM -> bf16 -> y ----
