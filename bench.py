@@ -313,6 +313,153 @@ def run_prefill(args):
     return 0
 
 
+SWEEPS = {
+    # name: (description, workload names from w3a16_gemv_b200.inputs.workloads())
+    "gemv4096": ("W3A16 GEMV M=1 N=4096 K=4096, codes uniform over 2..6, scales |N(0,0.02)|+1e-4",
+                 ("gemv_4096_m1",)),
+    "down": ("Llama-3.1-70B down_proj N=8192 K=28672 at M=1 and 8, GSQ 5-level codes, x with 1% outliers x20",
+             ("down_8192x28672_m1", "down_8192x28672_m8")),
+    "layer": ("Llama-3.1-70B layer at M=1: q, k, v, o, gate, up, down projections, codes uniform 0..7",
+              ("layer_q_proj_m1", "layer_k_proj_m1", "layer_v_proj_m1", "layer_o_proj_m1",
+               "layer_gate_proj_m1", "layer_up_proj_m1", "layer_down_proj_m1")),
+}
+
+
+def run_sweep(args):
+    """Per-call timing of the other decode configurations (one GPU): each call's weights rotate
+    among enough copies that every call streams them from HBM; for the layer sweep, also one CUDA
+    graph of the seven calls replayed `steps` times."""
+    import torch
+
+    from w3a16_gemv_b200 import build as wbuild
+    from w3a16_gemv_b200 import w3_check_device_error, w3_pack, w3a16_gemm
+    from w3a16_gemv_b200.inputs import workloads
+
+    world, rank, local = dist_setup()
+    if rank != 0:
+        return 0
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if not os.path.exists(wbuild.LIB):
+        wbuild.build()
+    desc, names = SWEEPS[args.workload]
+    wls = [workloads()[n] for n in names]
+    pass_bytes = sum(algorithmic_bytes(0, w.N, w.K) for w in wls)
+    copies = max(2, -(-3 * 126_000_000 // pass_bytes))  # more than three L2 sizes in rotation
+    calls = []
+    for w in wls:
+        p = w.problem()
+        packed = w3_pack(torch.from_numpy(p.codes).to(dev))
+        sc = torch.from_numpy(p.scales_bf16.view(np.int16)).view(torch.bfloat16).to(dev)
+        x = torch.from_numpy(p.x_bf16.view(np.int16)).view(torch.bfloat16).to(dev)
+        calls.append({"w": w, "packs": [packed] + [packed.clone() for _ in range(copies - 1)],
+                      "scales": [sc] + [sc.clone() for _ in range(copies - 1)], "x": x,
+                      "y": torch.empty((w.M, w.N), dtype=torch.bfloat16, device=dev)})
+    stream = torch.cuda.current_stream()
+
+    def one_pass(i, ev=None):
+        for j, c in enumerate(calls):
+            r = i % copies
+            if ev is not None:
+                ev[j][0].record(stream)
+            w3a16_gemm(c["x"], c["packs"][r], c["scales"][r], out=c["y"])
+            if ev is not None:
+                ev[j][1].record(stream)
+
+    for i in range(args.warmup):
+        one_pass(i)
+    torch.cuda.synchronize()
+    w3_check_device_error()
+    events = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)] for _ in calls]
+              for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.02)
+    torch.cuda.synchronize()
+    w0 = time.perf_counter()
+    for i in range(args.steps):
+        one_pass(args.warmup + i, events[i])
+    torch.cuda.synchronize()
+    w1 = time.perf_counter()
+    sampler.stop()
+    w3_check_device_error()
+    # device time per call without host overhead: a CUDA graph of the call on every weight copy, replayed
+    graph_us = []
+    reps = max(3, args.steps // copies)
+    for c in calls:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for r in range(copies):
+                w3a16_gemm(c["x"], c["packs"][r], c["scales"][r], out=c["y"])
+        g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            g.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        graph_us.append(a.elapsed_time(b) * 1e3 / (reps * copies))
+        del g
+    w3_check_device_error()
+    peak, peak_src = measured_peak()
+    out_calls, total_us, total_bytes = [], 0.0, 0
+    for j, c in enumerate(calls):
+        w = c["w"]
+        ts = np.array([events[i][j][0].elapsed_time(events[i][j][1]) for i in range(args.steps)]) * 1e3
+        med = float(np.median(ts))
+        b = algorithmic_bytes(w.M, w.N, w.K)
+        total_us += med
+        total_bytes += b
+        gu = graph_us[j]
+        out_calls.append({"name": w.name, "M": w.M, "N": w.N, "K": w.K,
+                          "us_median": med, "us_p10": float(np.percentile(ts, 10)),
+                          "us_p90": float(np.percentile(ts, 90)), "us_device_graph": gu,
+                          "GB/s": b / (gu * 1e-6) / 1e9, "frac_of_peak": b / (gu * 1e-6) / 1e9 / peak,
+                          "TFLOP/s": 2.0 * w.M * w.N * w.K / (gu * 1e-6) / 1e12})
+    line = {
+        "metric": METRIC, "value": total_bytes / (sum(graph_us) * 1e-6) / 1e9, "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sum(graph_us) / 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": desc, "calls": list(names),
+                   "l2": f"inputs larger than L2: {copies} rotating copies of every call's weights "
+                         f"({copies * pass_bytes / 1e6:.0f} MB)"},
+        "sum_of_median_us": total_us, "sum_of_device_us": sum(graph_us),
+        "timing": "us_median/p10/p90: CUDA events around each call (include host launch overhead when the "
+                  "kernel is shorter than it); us_device_graph and GB/s: one CUDA graph of the call on every "
+                  "weight copy, replayed, time per call",
+        "calls": out_calls, "peak": peak, "peak_source": peak_src,
+        "clocks": sampler.summary(w0, w1),
+    }
+    if args.workload == "layer":
+        # one CUDA graph of the seven calls on fixed copies, replayed
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            one_pass(0)  # warm the side stream outside the capture
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g):
+            one_pass(0)
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            g.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        w3_check_device_error()
+        g_us = a.elapsed_time(b) * 1e3 / args.steps
+        line["cuda_graph"] = {"us_per_replay": g_us, "GB/s": total_bytes / (g_us * 1e-6) / 1e9,
+                              "note": "weights of one copy, 7 calls per replay (L2 holds part of them)"}
+        del g
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_gpu(args):
     import torch
 
@@ -401,7 +548,9 @@ def run_gpu(args):
     for m in BATCHES:
         us = 1e3 * statistics.mean(per_call_ms[m])
         b = algorithmic_bytes(m, N_ROWS, K_COLS)
+        q = np.percentile(np.array(per_call_ms[m]) * 1e3, [10, 90])
         calls.append({"M": m, "us_mean": us, "us_median": 1e3 * statistics.median(per_call_ms[m]),
+                      "us_p10": float(q[0]), "us_p90": float(q[1]),
                       "GB/s": b / (us * 1e-6) / 1e9, "TFLOP/s": 2.0 * m * N_ROWS * K_COLS / (us * 1e-6) / 1e12,
                       "frac_of_peak": b / (us * 1e-6) / 1e9 / peak, "share": 0.0})
     tot = sum(c["us_mean"] for c in calls)
@@ -486,8 +635,9 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of CPU oracle work for cpu_baseline")
     ap.add_argument("--ref-budget", type=float, default=3.0, help="seconds of oracle work per reference step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=("gate_decode", "prefill"), default="gate_decode",
-                    help="gate_decode: the headline decode step (default); prefill: M=2048 tensor-core GEMM")
+    ap.add_argument("--workload", choices=("gate_decode", "prefill") + tuple(SWEEPS), default="gate_decode",
+                    help="gate_decode: the headline decode step (default); prefill: M=2048 tensor-core GEMM; "
+                         "gemv4096, down, layer: per-call timings of the other decode configurations")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -495,6 +645,8 @@ def main():
         return run_reference(args)
     if args.workload == "prefill":
         return run_prefill(args)
+    if args.workload in SWEEPS:
+        return run_sweep(args)
     return run_gpu(args)
 
 

@@ -95,12 +95,21 @@ __host__ __device__ constexpr int code_shift(int j) {
 
 constexpr uint32_t kMagic = 0x43004300u;  // bf16x2 (128.0, 128.0)
 
+// kMagic in a register the compiler cannot rematerialise: kernels create it once
+// and pass it to the unpack, which otherwise rebuilds the constant before many
+// of its LOP3s.
+__device__ __forceinline__ uint32_t pinned_magic() {
+    uint32_t m;
+    asm volatile("mov.b32 %0, %1;" : "=r"(m) : "n"(kMagic));
+    return m;
+}
+
 
 // Unpack one 96-bit block (w0, w1, w2) into the 16 bf16x2 pair registers.
 // Window s (a shift of the block by s bits) feeds the pairs whose codes sit at
 // window bits e_lo and 16 + e_hi.
-__device__ __forceinline__ void unpack_block(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t (&a)[16]) {
-    const uint32_t magic = kMagic;
+__device__ __forceinline__ void unpack_block(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t (&a)[16],
+                                             uint32_t magic = kMagic) {
     const uint32_t wm4 = w0 << 4;                     // s = -4
     const uint32_t w_2 = w0 >> 2;                     // s = 2
     const uint32_t w_8 = w0 >> 8;                     // s = 8
@@ -132,8 +141,7 @@ __device__ __forceinline__ void unpack_block(uint32_t w0, uint32_t w1, uint32_t 
 // that callers can interleave the unpack with the MMAs; with the index known at
 // compile time the windows shared by two pairs are computed once.
 template <int I>
-__device__ __forceinline__ uint32_t unpack_pair(uint32_t w0, uint32_t w1, uint32_t w2) {
-    const uint32_t magic = kMagic;
+__device__ __forceinline__ uint32_t unpack_pair(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t magic = kMagic) {
     if constexpr (I == 0) return and_or<pair_mask(4, 0)>(w0 << 4, magic);
     if constexpr (I == 1) return and_or<pair_mask(1, 3)>(w0 >> 2, magic);
     if constexpr (I == 2) return and_or<pair_mask(4, 0)>(w0 >> 2, magic);

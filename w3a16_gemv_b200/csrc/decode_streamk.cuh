@@ -85,22 +85,22 @@ __host__ __device__ __forceinline__ void warp_range(int64_t units, int w, int nw
 // the lane's two rows), unpacked right before the MMA.
 template <int K>
 __device__ __forceinline__ void tile_kstep(const uint32_t (&wa)[3], const uint32_t (&wb)[3], uint2 b,
-                                           float (&d)[4]) {
-    const uint32_t a0 = decode::unpack_pair<2 * K>(wa[0], wa[1], wa[2]);
-    const uint32_t a1 = decode::unpack_pair<2 * K>(wb[0], wb[1], wb[2]);
-    const uint32_t a2 = decode::unpack_pair<2 * K + 1>(wa[0], wa[1], wa[2]);
-    const uint32_t a3 = decode::unpack_pair<2 * K + 1>(wb[0], wb[1], wb[2]);
+                                           float (&d)[4], uint32_t magic) {
+    const uint32_t a0 = decode::unpack_pair<2 * K>(wa[0], wa[1], wa[2], magic);
+    const uint32_t a1 = decode::unpack_pair<2 * K>(wb[0], wb[1], wb[2], magic);
+    const uint32_t a2 = decode::unpack_pair<2 * K + 1>(wa[0], wa[1], wa[2], magic);
+    const uint32_t a3 = decode::unpack_pair<2 * K + 1>(wb[0], wb[1], wb[2], magic);
     mma_bf16_m16n8k16(d, a0, a1, a2, a3, b.x, b.y, d);
 }
 
 template <int K>
 __device__ __forceinline__ void block_ksteps(const uint32_t (&w)[4][3], const uint2 (&xs_g)[8],
-                                             float (&d0)[4], float (&d1)[4]) {
+                                             float (&d0)[4], float (&d1)[4], uint32_t magic) {
     if constexpr (K < 8) {
         const uint2 b = xs_g[K];
-        tile_kstep<K>(w[0], w[1], b, d0);
-        tile_kstep<K>(w[2], w[3], b, d1);
-        block_ksteps<K + 1>(w, xs_g, d0, d1);
+        tile_kstep<K>(w[0], w[1], b, d0, magic);
+        tile_kstep<K>(w[2], w[3], b, d1, magic);
+        block_ksteps<K + 1>(w, xs_g, d0, d1, magic);
     }
 }
 
@@ -111,7 +111,7 @@ template <int MT>
 __device__ __forceinline__ void block_group(const uint32_t *st, int pitch, int jstride, int j, int gabs,
                                             const uint2 *xs_lane, const float4 *ncorr,
                                             const uint16_t *const (&sc)[4], int r, int c,
-                                            float (&acc)[2][4]) {
+                                            float (&acc)[2][4], uint32_t magic) {
     uint32_t w[4][3];  // block c of the group in rows r, r+8, r+16, r+24
 #pragma unroll
     for (int h = 0; h < 4; ++h)
@@ -124,7 +124,7 @@ __device__ __forceinline__ void block_group(const uint32_t *st, int pitch, int j
     uint2 bfr[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) bfr[k] = xs_lane[(gabs * 8 + k) * MT * 4];
-    block_ksteps<0>(w, bfr, d0, d1);
+    block_ksteps<0>(w, bfr, d0, d1, magic);
     float s[4];
 #pragma unroll
     for (int h = 0; h < 4; ++h) s[h] = bf16_bits_to_f32(__ldg(sc[h] + gabs));
@@ -143,22 +143,22 @@ __device__ __forceinline__ void block_group(const uint32_t *st, int pitch, int j
 // latency of one chain is covered by the others.
 template <int K, int MT>
 __device__ __forceinline__ void stage_ksteps(const uint32_t (&w)[3][4][3], const uint2 *xs_g,
-                                             float (&d)[3][2][4]) {
+                                             float (&d)[3][2][4], uint32_t magic) {
     if constexpr (K < 8) {
 #pragma unroll
         for (int j = 0; j < 3; ++j) {
             const uint2 b = xs_g[(j * 8 + K) * MT * 4];
-            tile_kstep<K>(w[j][0], w[j][1], b, d[j][0]);
-            tile_kstep<K>(w[j][2], w[j][3], b, d[j][1]);
+            tile_kstep<K>(w[j][0], w[j][1], b, d[j][0], magic);
+            tile_kstep<K>(w[j][2], w[j][3], b, d[j][1], magic);
         }
-        stage_ksteps<K + 1, MT>(w, xs_g, d);
+        stage_ksteps<K + 1, MT>(w, xs_g, d, magic);
     }
 }
 
 template <int MT>
 __device__ __forceinline__ void full_stage(const uint32_t *st, int g, const uint2 *xs_lane, const float4 *ncorr,
                                            const uint16_t *const (&sc)[4], int r, int c,
-                                           float (&acc)[2][4]) {
+                                           float (&acc)[2][4], uint32_t magic) {
     float s[3][4];
 #pragma unroll
     for (int j = 0; j < 3; ++j)
@@ -183,7 +183,7 @@ __device__ __forceinline__ void full_stage(const uint32_t *st, int g, const uint
             d[j][t][3] = nc.w;
         }
     }
-    stage_ksteps<0, MT>(w, xs_lane + g * 8 * MT * 4, d);
+    stage_ksteps<0, MT>(w, xs_lane + g * 8 * MT * 4, d, magic);
 #pragma unroll
     for (int j = 0; j < 3; ++j)
 #pragma unroll
@@ -333,6 +333,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_sk_kernel(const __grid_
     float4 *slots = reinterpret_cast<float4 *>(smem + L.slot_off) + warp * 2 * 2 * 32;
 
     bool ok = true;
+    const uint32_t magic = decode::pinned_magic();
     uint32_t phase_bits = 0;
     float acc[2][4] = {};
     const uint16_t *sc[4] = {p.scales, p.scales, p.scales, p.scales};
@@ -362,10 +363,11 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_sk_kernel(const __grid_
         if (ok) {
             const uint32_t *st = reinterpret_cast<const uint32_t *>(ring + slot * kStageBytes);
             if (ng == kStageGroups) {
-                full_stage<MT>(st, cg, xs_lane, ncorr, sc, r, c, acc);
+                full_stage<MT>(st, cg, xs_lane, ncorr, sc, r, c, acc, magic);
             } else {
                 for (int j = 0; j < ng; ++j)
-                    block_group<MT>(st, kPitch1, kBlockRows * kPitch1, j, cg + j, xs_lane, ncorr, sc, r, c, acc);
+                    block_group<MT>(st, kPitch1, kBlockRows * kPitch1, j, cg + j, xs_lane, ncorr, sc, r, c, acc,
+                                    magic);
             }
         }
         // end of a segment: store a whole block, or park a partial one in a slot

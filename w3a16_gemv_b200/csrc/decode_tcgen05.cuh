@@ -178,6 +178,7 @@ static_assert(pair_kinds_complete(), "every pair's offsets are one of the five k
 // before every use.
 struct LevelConsts {
     uint32_t mul[kOffsetKinds], add[kOffsetKinds];
+    uint32_t magic = decode::pinned_magic();
     __device__ __forceinline__ LevelConsts() {
 #pragma unroll
         for (int k = 0; k < kOffsetKinds; ++k) {
@@ -246,7 +247,7 @@ __device__ __forceinline__ void half_levels(const uint32_t (&w)[kWordsPerGroup],
     for (int b = 0; b < 2; ++b) {
         const int bb = 2 * H + b;
         uint32_t blk[16];
-        decode::unpack_block(w[3 * bb], w[3 * bb + 1], w[3 * bb + 2], blk);
+        decode::unpack_block(w[3 * bb], w[3 * bb + 1], w[3 * bb + 2], blk, lc.magic);
 #pragma unroll
         for (int i = 0; i < 16; ++i) a[16 * b + i] = bf16x2_fma(blk[i], lc.mul[pair_kind(i)], lc.add[pair_kind(i)]);
     }
