@@ -71,6 +71,12 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         lib.oracle_gemm_f64_entries.restype = ctypes.c_int
         lib.oracle_weight_row_norms.argtypes = [p, p, i64, i64, p]
         lib.oracle_weight_row_norms.restype = ctypes.c_int
+        lib.oracle_ct4_words_per_row.argtypes = [i64]
+        lib.oracle_ct4_words_per_row.restype = i64
+        lib.oracle_pack_ct4.argtypes = [p, p, i64, i64]
+        lib.oracle_pack_ct4.restype = ctypes.c_int
+        lib.oracle_repack_ct4.argtypes = [p, p, i64, i64, p]
+        lib.oracle_repack_ct4.restype = ctypes.c_int
         if path is None:
             _lib = lib
         return lib
@@ -121,6 +127,28 @@ class Oracle:
         out = np.empty((N, K), dtype=np.uint8)
         _check(self.lib.oracle_unpack(_ptr(packed), _ptr(out), N, K), "oracle_unpack")
         return out
+
+    def ct4_words_per_row(self, K: int) -> int:
+        return int(self.lib.oracle_ct4_words_per_row(K))
+
+    def pack_ct4(self, codes: np.ndarray) -> np.ndarray:
+        """codes uint8 [N,K] (0..7) -> 4-bit container uint32 [N, K/8] (level + 8 per nibble, LSB first)."""
+        codes = _c(codes, np.uint8)
+        N, K = codes.shape
+        out = np.empty((N, max(self.ct4_words_per_row(K), 0)), dtype=np.uint32)
+        _check(self.lib.oracle_pack_ct4(_ptr(codes), _ptr(out), N, K), "oracle_pack_ct4")
+        return out
+
+    def repack_ct4(self, ct4: np.ndarray, K: int) -> tuple[np.ndarray, int]:
+        """4-bit container uint32 [N, K/8] -> (exact-width packed uint32 [N, 3K/32], levels clamped)."""
+        ct4 = _c(ct4.view(np.uint32), np.uint32)
+        N = ct4.shape[0]
+        if ct4.shape[1] != self.ct4_words_per_row(K):
+            raise ValueError("container width does not match K")
+        out = np.empty((N, max(self.words_per_row(K), 0)), dtype=np.uint32)
+        count = np.zeros(1, dtype=np.int64)
+        _check(self.lib.oracle_repack_ct4(_ptr(ct4), _ptr(out), N, K, _ptr(count)), "oracle_repack_ct4")
+        return out, int(count[0])
 
     def dequant_f32(self, packed: np.ndarray, scales_bf16: np.ndarray, K: int) -> np.ndarray:
         """W[n,k] = (c-4) * s[n,k//128] as fp32 [N,K] (exact)."""

@@ -199,3 +199,75 @@ int oracle_weight_row_norms(const uint32_t *packed, const uint16_t *scales,
     free(wrow);
     return 0;
 }
+
+/* ---- the 4-bit container written before the exact-width re-pack -------------------
+ *
+ * The card's note under "Storage layout" says that GSQ training first writes its
+ * shards in the compressed-tensors pack-quantized format, the 3-bit codebook
+ * padded into a 4-bit INT32 container, and that convert_to_humming.py re-packs
+ * them into the exact-width storage above.  The card does not print that
+ * container's layout.  Reading used here: eight 4-bit fields per int32 word,
+ * LSB first (level k of a row in bits 4*(k mod 8) .. 4*(k mod 8)+3 of word k/8),
+ * each field the signed level plus 8 (an unsigned nibble 0..15 for -8..7), so a
+ * row of K levels takes K/8 words.
+ */
+
+/* Container words per row: K levels x 4 bits / 32 bits per word. */
+int64_t oracle_ct4_words_per_row(int64_t K) {
+    if (K <= 0 || K % 8 != 0) return -1;
+    return K / 8;
+}
+
+/* codes [N,K] (0..7, level c - 4) -> container [N, K/8] words, fully written. */
+int oracle_pack_ct4(const uint8_t *codes, uint32_t *ct4, int64_t N, int64_t K) {
+    int64_t W = oracle_ct4_words_per_row(K);
+    if (!codes || !ct4 || N < 0 || W < 0) return -1;
+    for (int64_t n = 0; n < N; ++n) {
+        uint32_t *row = ct4 + n * W;
+        for (int64_t w = 0; w < W; ++w) row[w] = 0;
+        for (int64_t k = 0; k < K; ++k) {
+            unsigned c = codes[n * K + k];
+            if (c > 7) return -1;
+            int q = (int)c - 4;
+            unsigned field = (unsigned)(q + 8);
+            for (int i = 0; i < 4; ++i) {
+                int64_t b = 4 * k + i;
+                row[b / 32] |= ((field >> i) & 1u) << (b % 32);
+            }
+        }
+    }
+    return 0;
+}
+
+/* container [N, K/8] -> exact-width packed [N, 3K/32].  A level outside -4..3 has
+ * no 3-bit code: it is clamped to the nearer of -4 and 3, and the number of such
+ * levels is written to *out_of_range. */
+int oracle_repack_ct4(const uint32_t *ct4, uint32_t *packed, int64_t N, int64_t K, int64_t *out_of_range) {
+    int64_t W4 = oracle_ct4_words_per_row(K), W3 = oracle_words_per_row(K);
+    if (!ct4 || !packed || !out_of_range || N < 0 || W4 < 0 || W3 < 0) return -1;
+    *out_of_range = 0;
+    for (int64_t n = 0; n < N; ++n) {
+        const uint32_t *in = ct4 + n * W4;
+        uint32_t *out = packed + n * W3;
+        for (int64_t w = 0; w < W3; ++w) out[w] = 0;
+        for (int64_t k = 0; k < K; ++k) {
+            unsigned field = 0;
+            for (int i = 0; i < 4; ++i)
+                field |= stream_bit(in, 4 * k + i) << i;
+            int q = (int)field - 8;
+            if (q < -4) {
+                q = -4;
+                ++*out_of_range;
+            } else if (q > 3) {
+                q = 3;
+                ++*out_of_range;
+            }
+            unsigned c = (unsigned)(q + 4);
+            for (int i = 0; i < 3; ++i) {
+                int64_t b = 3 * k + i;
+                out[b / 32] |= ((c >> i) & 1u) << (b % 32);
+            }
+        }
+    }
+    return 0;
+}

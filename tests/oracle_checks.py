@@ -232,6 +232,36 @@ def check_rejects_bad_arguments(orc):
         raise AssertionError("a code of 8 was accepted")
 
 
+def check_ct4_container_words(orc):
+    """The 4-bit container pins: hand-derived words for packing and for the re-pack with clamping."""
+    g = load_golden("ct4_container_words.json")
+    for case in g["pack_cases"]:
+        codes = np.full((1, 128), 4, dtype=np.uint8)  # level 0 everywhere
+        for pos, level in case["levels"].items():
+            codes[0, int(pos)] = level + 4
+        words = orc.pack_ct4(codes)
+        assert words.shape == (1, 16), case["name"]
+        assert int(words[0, 0]) == int(case["word"], 16), case["name"]
+        assert np.all(words[0, 1:] == 0x88888888), case["name"]
+    for case in g["repack_cases"]:
+        ct4 = np.full((1, 16), 0x88888888, dtype=np.uint32)
+        ct4[0, 0] = int(case["word"], 16)
+        packed, clamped = orc.repack_ct4(ct4, 128)
+        codes = orc.unpack(packed, 128)
+        assert list(codes[0, :8]) == case["codes"], case["name"]
+        assert np.all(codes[0, 8:] == 4), case["name"]
+        assert clamped == case["out_of_range"], case["name"]
+
+
+def check_ct4_repack_equals_direct_pack(orc):
+    """Re-packing the container of any codes gives the exact-width words of the same codes."""
+    rng = np.random.Generator(np.random.PCG64(7))
+    codes = rng.integers(0, 8, size=(5, 384), dtype=np.uint8)
+    packed, clamped = orc.repack_ct4(orc.pack_ct4(codes), 384)
+    assert clamped == 0
+    assert np.array_equal(packed, orc.pack(codes))
+
+
 ALL_CHECKS = [
     check_worked_example_shapes,
     check_bits_per_weight,
@@ -246,4 +276,6 @@ ALL_CHECKS = [
     check_numpy_cross_check,
     check_weight_row_norms,
     check_rejects_bad_arguments,
+    check_ct4_container_words,
+    check_ct4_repack_equals_direct_pack,
 ]

@@ -28,6 +28,11 @@ MUTANTS = [
     ("scale_not_applied_in_product",
      "wrow[k] = (float)q * bf16_bits_to_float(scales[n * G + k / ORACLE_GROUP]);", "wrow[k] = (float)q;", 1),
     ("words_per_row_4bit_container", "return K * 3 / 32;", "return K * 4 / 32;", 1),
+    ("ct4_level_offset_7", "int q = (int)field - 8;", "int q = (int)field - 7;", 1),
+    ("ct4_field_bits_msb_first", "field |= stream_bit(in, 4 * k + i) << i;",
+     "field |= stream_bit(in, 4 * k + i) << (3 - i);", 1),
+    ("ct4_clamp_not_counted", "                q = 3;\n                ++*out_of_range;", "                q = 3;", 1),
+    ("ct4_pack_offset_7", "unsigned field = (unsigned)(q + 8);", "unsigned field = (unsigned)(q + 7);", 1),
 ]
 
 
