@@ -91,6 +91,24 @@ w3_status w3_pack(const uint8_t *codes, int32_t *packed, int64_t N, int64_t K, w
 w3_status w3_unpack(const int32_t *packed, uint8_t *codes, int64_t N, int64_t K, w3_stream_t stream);
 
 /*
+ * w3_repack_ct4 -- 4-bit container [N, K/8] int32 -> packed [N, 3K/32] int32 in
+ * the exact-width format above.  The card's note under "Storage layout" says
+ * GSQ training first writes shards in the compressed-tensors pack-quantized
+ * format, the 3-bit codebook padded into a 4-bit INT32 container, and that
+ * convert_to_humming.py re-packs them into the exact-width storage; it prints
+ * no container layout.  Layout read here: eight 4-bit fields per int32, LSB
+ * first (level k of a row in bits 4*(k%8)..4*(k%8)+3 of word k/8), each field
+ * the signed level plus 8.  A level outside -4..3 has no 3-bit code: it is
+ * clamped to -4 or 3, and if `out_of_range` (a device int64, 8-byte aligned)
+ * is not NULL the call sets it to the number of clamped levels (stream-
+ * ordered).  Scales are unchanged by the re-pack.  Errors: W3_ERR_NULL,
+ * W3_ERR_SHAPE (N < 1, K not a positive multiple of 128), W3_ERR_ALIGN,
+ * W3_ERR_ALIAS, W3_ERR_UNSUPPORTED, W3_ERR_CUDA.
+ */
+w3_status w3_repack_ct4(const int32_t *ct4, int32_t *packed, int64_t N, int64_t K, int64_t *out_of_range,
+                        w3_stream_t stream);
+
+/*
  * w3_dequant_f32 -- w[n,k] = (c[n,k] - 4) * scales[n, k/128] as fp32 [N,K].
  * The symmetric group-wise dequantization of the card's quantization_config
  * (weight_scale_type "group", weight_scale_group_size 128, has_zero_point

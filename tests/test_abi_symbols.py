@@ -63,6 +63,12 @@ def test_host_argument_checks(lib):
     assert lib.w3_pack(FAKE_A, FAKE_A, 4, 128, NULL) == 7
     assert lib.w3_unpack(FAKE_A, NULL, 4, 128, NULL) == 1
     assert lib.w3_dequant_f32(FAKE_A, FAKE_B, FAKE_C, 4, 130, NULL) == 2
+    r = lib.w3_repack_ct4
+    assert r(NULL, FAKE_B, 4, 128, NULL, NULL) == 1  # W3_ERR_NULL
+    assert r(FAKE_A, FAKE_B, 4, 96, NULL, NULL) == 2  # K % 128
+    assert r(FAKE_A + 4, FAKE_B, 4, 128, NULL, NULL) == 3  # misaligned container
+    assert r(FAKE_A, FAKE_B, 4, 128, FAKE_C + 4, NULL) == 3  # misaligned counter
+    assert r(FAKE_A, FAKE_A + 16, 4, 128, NULL, NULL) == 7  # output overlaps the container
 
 
 def test_no_silent_fallback_without_a_device(lib):

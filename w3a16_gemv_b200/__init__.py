@@ -17,6 +17,7 @@ from ._binding import (  # noqa: F401
     w3_groups_per_row,
     w3_pack,
     w3_packed_words_per_row,
+    w3_repack_ct4,
     w3_unpack,
     w3a16_gemm,
     w3a16_gemm_noalloc,
@@ -31,6 +32,7 @@ __all__ = [
     "w3_groups_per_row",
     "w3_pack",
     "w3_packed_words_per_row",
+    "w3_repack_ct4",
     "w3_unpack",
     "w3a16_gemm",
     "w3a16_gemm_noalloc",

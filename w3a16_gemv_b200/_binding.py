@@ -40,6 +40,7 @@ SIGNATURES = [
     ("w3_pack", ctypes.c_int, [_P, _P, _I64, _I64, _P]),
     ("w3_unpack", ctypes.c_int, [_P, _P, _I64, _I64, _P]),
     ("w3_dequant_f32", ctypes.c_int, [_P, _P, _P, _I64, _I64, _P]),
+    ("w3_repack_ct4", ctypes.c_int, [_P, _P, _I64, _I64, _P, _P]),
     ("w3a16_gemm", ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P]),
     ("w3a16_gemm_noalloc", ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P]),
     ("w3_check_device_error", ctypes.c_int, [_P]),
@@ -132,6 +133,25 @@ def w3_unpack(packed: torch.Tensor, K: int, codes: torch.Tensor | None = None, s
     _need(codes, torch.uint8, "codes")
     _check(lib().w3_unpack(packed.data_ptr(), codes.data_ptr(), N, K, _stream(stream)), "w3_unpack")
     return codes
+
+
+def w3_repack_ct4(ct4: torch.Tensor, K: int, packed: torch.Tensor | None = None, count_out_of_range: bool = False,
+                  stream=None):
+    """4-bit container int32 [N, K/8] -> exact-width packed int32 [N, 3K/32].
+
+    With count_out_of_range, returns (packed, count) where count is a device int64 tensor holding the
+    number of levels outside -4..3 that were clamped."""
+    _need(ct4, torch.int32, "ct4")
+    N = ct4.shape[0]
+    if ct4.dim() != 2 or ct4.shape[1] * 8 != K:
+        raise ValueError("ct4 must be [N, K/8]")
+    if packed is None:
+        packed = torch.empty((N, w3_packed_words_per_row(K)), dtype=torch.int32, device=ct4.device)
+    _need(packed, torch.int32, "packed")
+    count = torch.zeros(1, dtype=torch.int64, device=ct4.device) if count_out_of_range else None
+    _check(lib().w3_repack_ct4(ct4.data_ptr(), packed.data_ptr(), N, K, count.data_ptr() if count is not None else None,
+                               _stream(stream)), "w3_repack_ct4")
+    return (packed, count) if count_out_of_range else packed
 
 
 def w3_dequant_f32(packed: torch.Tensor, scales: torch.Tensor, K: int, out: torch.Tensor | None = None,

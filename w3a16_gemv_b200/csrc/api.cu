@@ -431,6 +431,26 @@ w3_status w3_unpack(const int32_t *packed, uint8_t *codes, int64_t N, int64_t K,
     return launch_status();
 }
 
+w3_status w3_repack_ct4(const int32_t *ct4, int32_t *packed, int64_t N, int64_t K, int64_t *out_of_range,
+                        w3_stream_t stream) {
+    if (!ct4 || !packed) return W3_ERR_NULL;
+    if (w3_status s = check_nk(N, K)) return s;
+    if (!aligned16(ct4) || !aligned16(packed) || (out_of_range && (reinterpret_cast<uintptr_t>(out_of_range) & 7u)))
+        return W3_ERR_ALIGN;
+    if (overlaps(ct4, N * K / 2, packed, N * K * 3 / 8) ||
+        (out_of_range && (overlaps(out_of_range, 8, ct4, N * K / 2) || overlaps(out_of_range, 8, packed, N * K * 3 / 8))))
+        return W3_ERR_ALIAS;
+    int sms;
+    if (w3_status s = device_setup(&sms)) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (out_of_range && cudaMemsetAsync(out_of_range, 0, sizeof(int64_t), st) != cudaSuccess) return W3_ERR_CUDA;
+    const int64_t nblocks = N * K / 32;
+    repack_ct4_kernel<<<grid_for(nblocks, 256), 256, 0, st>>>(reinterpret_cast<const uint4 *>(ct4),
+                                                             reinterpret_cast<uint32_t *>(packed), nblocks,
+                                                             reinterpret_cast<unsigned long long *>(out_of_range));
+    return launch_status();
+}
+
 w3_status w3_dequant_f32(const int32_t *packed, const uint16_t *scales, float *w, int64_t N, int64_t K,
                          w3_stream_t stream) {
     if (!packed || !scales || !w) return W3_ERR_NULL;

@@ -75,3 +75,43 @@ inline unsigned grid_for(int64_t nblocks, int threads) {
 }
 
 }  // namespace w3
+
+namespace w3 {
+
+// Re-pack from the 4-bit container GSQ training writes before the exact-width
+// storage (the card's note under "Storage layout": compressed-tensors
+// pack-quantized, the 3-bit codebook padded into a 4-bit INT32 container,
+// re-packed by convert_to_humming.py).  The container layout is a reading (the
+// card prints none): eight 4-bit fields per word, LSB first, each the level
+// plus 8.  A 32-level block is 4 container words (16 bytes) in, 3 words out.
+// Levels outside -4..3 have no 3-bit code: they are clamped to -4 or 3 and
+// counted into *out_of_range (when given).
+__global__ void __launch_bounds__(256) repack_ct4_kernel(const uint4 *__restrict__ ct4, uint32_t *__restrict__ packed,
+                                                         int64_t nblocks, unsigned long long *out_of_range) {
+    const int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    unsigned clamped = 0;
+    if (b < nblocks) {
+        const uint4 q = ct4[b];
+        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+        unsigned __int128 v = 0;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            int level = static_cast<int>((w[j >> 3] >> (4 * (j & 7))) & 15u) - 8;
+            if (level < -4 || level > 3) {
+                ++clamped;
+                level = level < -4 ? -4 : 3;
+            }
+            v |= static_cast<unsigned __int128>(level + 4) << (3 * j);
+        }
+        uint32_t *dst = packed + 3 * b;
+        dst[0] = static_cast<uint32_t>(v);
+        dst[1] = static_cast<uint32_t>(v >> 32);
+        dst[2] = static_cast<uint32_t>(v >> 64);
+    }
+    if (out_of_range) {
+        clamped = __reduce_add_sync(0xffffffffu, clamped);
+        if ((threadIdx.x & 31) == 0 && clamped) atomicAdd(out_of_range, static_cast<unsigned long long>(clamped));
+    }
+}
+
+}  // namespace w3
