@@ -456,8 +456,70 @@ def run_sweep(args):
         line["cuda_graph"] = {"us_per_replay": g_us, "GB/s": total_bytes / (g_us * 1e-6) / 1e9,
                               "note": "weights of one copy, 7 calls per replay (L2 holds part of them)"}
         del g
+        line["fused"] = fused_layer(calls, copies, args, stream, total_bytes)
     print(json.dumps(line), flush=True)
     return 0
+
+
+def fused_layer(calls, copies, args, stream, total_bytes):
+    """The same layer as 4 calls: q, k, v and gate, up concatenated along N (rows of the format
+    are independent, so a row-concatenated packed/scales pair is one weight), o and down alone.
+    Device time of each call from graph replays over its copies, and one graph of the 4 calls."""
+    import torch
+
+    from w3a16_gemv_b200 import w3_check_device_error, w3a16_gemm
+
+    by = {c["w"].name: c for c in calls}
+
+    def cat(names):
+        cs = [by[n] for n in names]
+        return {"name": "+".join(n.split("_")[1] for n in names), "M": 1,
+                "N": sum(c["w"].N for c in cs), "K": cs[0]["w"].K, "x": cs[0]["x"],
+                "packs": [torch.cat([c["packs"][r] for c in cs]) for r in range(copies)],
+                "scales": [torch.cat([c["scales"][r] for c in cs]) for r in range(copies)]}
+
+    fcalls = [cat(["layer_q_proj_m1", "layer_k_proj_m1", "layer_v_proj_m1"]), cat(["layer_o_proj_m1"]),
+              cat(["layer_gate_proj_m1", "layer_up_proj_m1"]), cat(["layer_down_proj_m1"])]
+    for c in fcalls:
+        c["y"] = torch.empty((1, c["N"]), dtype=torch.bfloat16, device=c["x"].device)
+    reps = max(3, args.steps // copies)
+    out = []
+    for c in fcalls:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for r in range(copies):
+                w3a16_gemm(c["x"], c["packs"][r], c["scales"][r], out=c["y"])
+        g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            g.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        us = a.elapsed_time(b) * 1e3 / (reps * copies)
+        byt = algorithmic_bytes(1, c["N"], c["K"])
+        out.append({"name": c["name"], "N": c["N"], "K": c["K"], "us_device_graph": us,
+                    "GB/s": byt / (us * 1e-6) / 1e9})
+        del g
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for c in fcalls:
+            w3a16_gemm(c["x"], c["packs"][0], c["scales"][0], out=c["y"])
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.steps):
+        g.replay()
+    b.record(stream)
+    torch.cuda.synchronize()
+    w3_check_device_error()
+    g_us = a.elapsed_time(b) * 1e3 / args.steps
+    del g
+    return {"calls": out, "sum_of_device_us": sum(c["us_device_graph"] for c in out),
+            "cuda_graph_us_per_replay": g_us, "GB/s": total_bytes / (g_us * 1e-6) / 1e9}
 
 
 def run_gpu(args):

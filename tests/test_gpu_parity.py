@@ -131,6 +131,28 @@ def test_position_probe(orc):
         assert np.all(np.abs(y - want) <= 2.0 ** -8 * np.abs(want) + 1e-30), k0
 
 
+def test_row_concatenated_weights_are_one_weight(orc):
+    """q, k, v weights concatenated along N run as one call: each part of the result is within
+    the bound of the oracle of its own weight (the format's rows are independent)."""
+    K = 2048
+    parts = [make_problem(1, n, K, "uniform8", "lognormal", "normal", seed=40 + i) for i, n in enumerate((768, 256, 256))]
+    x, _, _ = device_problem(parts[0])
+    packs, scs = [], []
+    for p in parts:
+        _, codes, scales = device_problem(p)
+        packs.append(w3_pack(codes))
+        scs.append(scales)
+    y = from_dev_bf16(w3a16_gemm(x, torch.cat(packs), torch.cat(scs)))
+    w3_check_device_error()
+    n0 = 0
+    for p in parts:
+        ref_packed = orc.pack(p.codes)
+        ref = orc.gemm_f64(parts[0].x_bf16, ref_packed, p.scales_bf16)
+        tol = bound(parts[0].x_bf16, orc.weight_row_norms(ref_packed, p.scales_bf16, K), K)
+        assert_within_bound(y[:, n0:n0 + p.N], ref, tol, f"part N={p.N}")
+        n0 += p.N
+
+
 def _sampled_check(orc, name, n_samples=1024, seed=0):
     wl = workloads()[name]
     p = wl.problem()

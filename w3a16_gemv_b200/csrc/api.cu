@@ -28,6 +28,10 @@
 #define W3_PREFILL_TCGEN05 1
 #endif
 // Smallest decode batch that uses the tcgen05 decode kernel (above 16: never).
+// Launch the decode kernels with programmatic dependent launch.
+#ifndef W3_DECODE_PDL
+#define W3_DECODE_PDL 1
+#endif
 #ifndef W3_DECODE_TC_MIN_M
 #define W3_DECODE_TC_MIN_M 5
 #endif
@@ -135,6 +139,16 @@ PFN_cuTensorMapEncodeTiled tensor_map_encoder() {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Programmatic dependent launch: the kernel may start before the previous kernel in
+// the stream ends; it waits for it (griddepcontrol.wait) before touching x, y or
+// scratch.  Weights and scales are read before that wait, so a kernel that writes
+// them must not precede the call with an early trigger of its own (this library's
+// kernels that write weights -- pack, repack -- never trigger early).
+void set_pdl(cudaLaunchAttribute &a) {
+    a.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    a.val.programmaticStreamSerializationAllowed = 1;
+}
+
 bool overlaps(const void *a, int64_t abytes, const void *b, int64_t bbytes) {
     const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
     return a0 < b0 + static_cast<uintptr_t>(bbytes) && b0 < a0 + static_cast<uintptr_t>(abytes);
@@ -191,6 +205,10 @@ w3_status launch_decode_sk(const uint16_t *x, const int32_t *packed, const uint1
     cfg.blockDim = dim3(decode_sk::kWarps * 32, 1, 1);
     cfg.dynamicSmemBytes = P.smem_bytes;
     cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    set_pdl(attr[0]);  // overlaps the set-up with the previous kernel's tail
+    cfg.attrs = attr;
+    cfg.numAttrs = W3_DECODE_PDL ? 1 : 0;
     cudaError_t e;
     switch (P.mt) {
         case 1: e = cudaLaunchKernelEx(&cfg, decode_sk::decode_sk_kernel<1>, prm); break;
@@ -242,6 +260,10 @@ w3_status launch_decode_tc(const uint16_t *x, const int32_t *packed, const uint1
     cfg.blockDim = dim3(decode_tc::kThreads, 1, 1);
     cfg.dynamicSmemBytes = decode_tc::SmemLayout::total;
     cfg.stream = stream;
+    cudaLaunchAttribute mattr[1];
+    set_pdl(mattr[0]);
+    cfg.attrs = mattr;
+    cfg.numAttrs = W3_DECODE_PDL ? 1 : 0;
     if (cudaLaunchKernelEx(&cfg, decode_tc::decode_tc_kernel, prm) != cudaSuccess) return W3_ERR_CUDA;
     if (P.P == 1) return W3_OK;
     decode_tc::FixupParams fp;
@@ -257,8 +279,7 @@ w3_status launch_decode_tc(const uint16_t *x, const int32_t *packed, const uint1
     fcfg.blockDim = dim3(decode_tc::kRows, 1, 1);
     fcfg.stream = stream;
     cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    set_pdl(attr[0]);
     fcfg.attrs = attr;
     fcfg.numAttrs = 1;
     return cudaLaunchKernelEx(&fcfg, decode_tc::decode_tc_fixup_kernel, fp) == cudaSuccess ? W3_OK : W3_ERR_CUDA;

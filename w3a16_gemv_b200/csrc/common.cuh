@@ -120,6 +120,16 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
         : "memory");
 }
 
+// ---- programmatic dependent launch ---------------------------------------------------
+// A kernel launched with programmatic stream serialization may start while the
+// previous kernel in the stream is still running.  It signals its own dependents
+// early (pdl_trigger) and waits for its predecessor's completion and memory
+// (pdl_wait) before it reads anything the predecessor may write (x) or writes
+// anything it may read (y, scratch).  Both are no-ops for a normal launch.
+
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---- thread-block clusters ---------------------------------------------------------
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {

@@ -220,6 +220,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_sk_kernel(const __grid_
     const int lane = threadIdx.x & 31;
     const int r = lane >> 2;
     const int c = lane & 3;
+    pdl_trigger();  // the next kernel in the stream may start its own set-up
 
     const int NB = (N + kBlockRows - 1) / kBlockRows;
     const int b_begin = static_cast<int>(static_cast<int64_t>(NB) * blockIdx.x / p.ctas);
@@ -305,6 +306,9 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_sk_kernel(const __grid_
         advance(ibl, ig, issue(ibl, ig, issue_slot));
         issue_slot = (issue_slot + 1 == depth) ? 0 : issue_slot + 1;
     }
+    // x (and, at the end, y) may belong to the previous kernel in the stream: wait for it here,
+    // after the first weight stages are already in flight
+    pdl_wait();
     decode::Params dp;  // prepare_x reads x, M and K only
     dp.x = p.x;
     dp.M = M;

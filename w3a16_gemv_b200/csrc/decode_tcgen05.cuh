@@ -320,7 +320,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_tc_kernel(const _
     const int lane = threadIdx.x & 31;
 
     // the partial-sum fix-up grid may start now; it waits for this grid to finish
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    pdl_trigger();
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -343,6 +343,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_tc_kernel(const _
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     bool ok = true;
+    // x, y and the scratch may belong to the previous kernel in the stream
+    pdl_wait();
 
     if (warp == 0) {
         // ---- loads, then the in-place permutation of x one stage behind ----
@@ -567,7 +569,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_tc_kernel(const _
 // falls inside (when it is the first such boundary of that tile) and adds the
 // partial sums of the CTAs that cover it, in CTA order.
 __global__ void __launch_bounds__(kRows) decode_tc_fixup_kernel(const __grid_constant__ FixupParams p) {
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+    pdl_wait();
     const int i = blockIdx.x + 1;
     const int64_t u = unit_begin(i, p.U, p.P);
     const int64_t t = u / p.G;
