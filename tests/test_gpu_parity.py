@@ -50,6 +50,8 @@ SMALL = [
     (256, 256, 256, "uniform8", "lognormal", "normal"),
     (300, 1000, 1024, "gsq_5level", "absnormal", "normal_outliers"),
     (513, 200, 384, "uniform8", "lognormal", "normal"),
+    (32, 28672, 1024, "uniform8", "lognormal", "normal"),   # 128 tiles at once: packed-word buffer reuse
+    (32, 448, 8192, "gsq_5level", "absnormal", "normal"),   # 32 packed-word copies per tile
 ]
 
 

@@ -299,6 +299,12 @@ w3_status launch_prefill(const uint16_t *x, const int32_t *packed, const uint16_
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return W3_ERR_CUDA;
+    if (W3_PREFILL_WTMA) {
+        // [BN rows][24 words] boxes over the packed matrix: four stages of the CTA's rows per copy
+        if (encode_packed_map(&prm.tmap_w, packed, N, static_cast<int64_t>(K) * 3 / 32,
+                              prefill::kChunkStages * prefill::kStageWords, static_cast<uint32_t>(P.tile_n)) != W3_OK)
+            return W3_ERR_CUDA;
+    }
     prm.packed = reinterpret_cast<const uint32_t *>(packed);
     prm.scales = scales;
     prm.y = y;
@@ -501,7 +507,8 @@ w3_status w3a16_gemm(const uint16_t *x, const int32_t *packed, const uint16_t *s
     cudaMemPool_t pool;
     if (w3_status s = device_setup(&sms, &pool)) return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (M > 16 && W3_PREFILL_TCGEN05)
+    // the prefill kernel's packed-word copies are 24 words wide: rows of at least 256 codes
+    if (M > 16 && W3_PREFILL_TCGEN05 && K >= 256)
         return launch_prefill(x, packed, scales, y, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), sms,
                               st);
     // The tensor-core decode for N >= 256: one call per 16 batch rows, all sharing

@@ -40,7 +40,14 @@ constexpr int kMaxTileN = 256;       // rows of W per CTA at most
 constexpr int kStageK = 64;          // k per pipeline stage = one 128-byte swizzle atom of bf16
 constexpr int kStages = 3;
 constexpr int kDequantWarps = 8;     // one W row per thread: BN <= 256
-constexpr int kThreads = (2 + kDequantWarps) * 32;
+// 1: the packed words reach shared memory by TMA ([BN rows][24 words], four
+// stages per copy, from a producer warp) and each thread copies its row into
+// registers; 0: each thread loads its row's words from global memory.
+#ifndef W3_PREFILL_WTMA
+#define W3_PREFILL_WTMA 1
+#endif
+constexpr int kChunkStages = 4;                   // stages per packed-word copy
+constexpr int kThreads = (2 + kDequantWarps + (W3_PREFILL_WTMA ? 1 : 0)) * 32;
 constexpr int kTmemCols = 512;
 constexpr int kABytes = kUmmaM * kStageK * 2;     // 16 KB per 128-row tile and stage
 constexpr int kBBytes = kMaxTileN * kStageK * 2;  // 32 KB per stage (BN rows used)
@@ -54,13 +61,16 @@ struct SmemLayout {
     // all operand buffers are 1024-byte aligned (the 128-byte swizzle period)
     static constexpr int a_off = 0;                                  // [kStages][2][kABytes]
     static constexpr int b_off = a_off + kStages * 2 * kABytes;      // [kStages][kBBytes]
-    static constexpr int bar_off = b_off + kStages * kBBytes;        // u64 full_a, full_b, empty [kStages], acc
-    static constexpr int tmem_slot_off = bar_off + (3 * kStages + 1) * 8;
+    static constexpr int w_off = b_off + kStages * kBBytes;          // [BN rows][24 words] packed
+    static constexpr int sink_off = w_off + kMaxTileN * kChunkStages * 6 * 4;  // u32 [256]: see the release below
+    static constexpr int bar_off = sink_off + kMaxTileN * 4;         // full_a, full_b, empty [kStages], acc, w_full, w_empty
+    static constexpr int tmem_slot_off = bar_off + (3 * kStages + 3) * 8;
     static constexpr int total = tmem_slot_off + 16 + 1024;          // + slack to align the base to 1024
 };
 
 struct Params {
     CUtensorMap tmap_x;  // x [M][K] bf16, box [128 rows][64 k], 128-byte swizzle
+    CUtensorMap tmap_w;  // packed [N][3K/32] u32, box [BN rows][24 words]
     const uint32_t *packed;
     const uint16_t *scales;
     uint16_t *y;
@@ -177,6 +187,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     const uint32_t bar_full_b = bar_full_a + 8 * kStages;
     const uint32_t bar_empty = bar_full_b + 8 * kStages;
     const uint32_t bar_acc = bar_empty + 8 * kStages;
+    const uint32_t bar_wfull = bar_acc + 8, bar_wempty = bar_acc + 16;
+    constexpr int kChunkWords = kChunkStages * kStageWords;  // 24 words per row and copy
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + SmemLayout::tmem_slot_off);
 
     const int warp = threadIdx.x >> 5;
@@ -185,7 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     const int n0 = blockIdx.x * p.tile_n;
     const int nstages = p.K / kStageK;
     const int G = p.K / kGroup;
-    const int W = G * kWordsPerGroup;
+    [[maybe_unused]] const int W = G * kWordsPerGroup;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -194,6 +206,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             mbar_init(bar_empty + 8 * s, 1);
         }
         mbar_init(bar_acc, 1);
+        mbar_init(bar_wfull, 1);
+        mbar_init(bar_wempty, kDequantWarps * 32);
         mbar_init_fence();
     }
     if (warp == 1) {  // allocate the accumulators
@@ -246,13 +260,105 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             umma_commit(bar_empty + 8 * slot);  // frees the stage once these MMAs have read it
         }
         if (ok) umma_commit(bar_acc);  // all accumulation done
+    } else if (warp == 2 + kDequantWarps) {
+        // ---- packed words of the CTA's rows, four stages per TMA copy ----
+        if (lane == 0) {
+            const int nchunks = (nstages + kChunkStages - 1) / kChunkStages;
+            for (int c = 0; c < nchunks && ok; ++c) {
+                ok = mbar_wait_bounded(bar_wempty, (c & 1) ^ 1);
+                if (!ok) break;
+                mbar_arrive_expect_tx(bar_wfull, p.tile_n * kChunkWords * 4);
+                tma_load_2d(sbase + SmemLayout::w_off, &p.tmap_w, c * kChunkWords, n0, bar_wfull);
+            }
+        }
     } else {
         // ---- B producers: dequantize one W row per thread ----
         const int t = threadIdx.x - 64;  // 0..255
         const int n = n0 + t;
         const bool row_ok = (t < p.tile_n) && (n < p.N);
+#if !W3_PREFILL_WTMA
         const uint32_t *prow = p.packed + static_cast<int64_t>(row_ok ? n : 0) * W;
+#endif
         const uint16_t *srow = p.scales + static_cast<int64_t>(row_ok ? n : 0) * G;
+#if W3_PREFILL_WTMA
+        // the row's 24 words of a 4-stage chunk come from the shared-memory copy; the chunk's two
+        // group scales are loaded one chunk ahead
+        const uint32_t *wsm = reinterpret_cast<const uint32_t *>(smem + SmemLayout::w_off);
+        const int nchunks = (nstages + kChunkStages - 1) / kChunkStages;
+        uint32_t sc_cur[2] = {0u, 0u}, sc_next[2] = {0u, 0u};
+        auto load_scales = [&](int c, uint32_t (&dst)[2]) {
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const int g = 2 * c + i;
+                const uint32_t hs = (row_ok && g < G) ? __ldg(srow + g) : 0u;
+                dst[i] = hs | (hs << 16);
+            }
+        };
+        load_scales(0, sc_cur);
+        for (int c = 0; c < nchunks && ok; ++c) {
+            load_scales(c + 1, sc_next);
+            ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar_wfull, c & 1));
+            if (!ok) break;
+            uint32_t words[kChunkWords];
+            if (t < p.tile_n) {
+                const uint4 *src = reinterpret_cast<const uint4 *>(wsm + t * kChunkWords);
+#pragma unroll
+                for (int i = 0; i < kChunkWords / 4; ++i) {
+                    const uint4 q = src[i];
+                    words[4 * i] = q.x;
+                    words[4 * i + 1] = q.y;
+                    words[4 * i + 2] = q.z;
+                    words[4 * i + 3] = q.w;
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < kChunkWords; ++i) words[i] = 0u;
+            }
+            // The next copy into the buffer is an async-proxy write, and the arrive below orders
+            // memory operations, not the arrival of load results in registers.  A store that
+            // depends on every loaded register therefore precedes the arrive: the buffer is
+            // released only once the loads have completed.
+            uint32_t landed = 0;
+#pragma unroll
+            for (int i = 0; i < kChunkWords; i += 4) landed ^= words[i];
+            asm volatile("st.shared.u32 [%0], %1;" ::"r"(sbase + SmemLayout::sink_off + 4 * t), "r"(landed) : "memory");
+            mbar_arrive(bar_wempty);
+#pragma unroll
+            for (int u = 0; u < kChunkStages; ++u) {
+                const int s = c * kChunkStages + u;
+                if (s >= nstages || !ok) break;
+                uint32_t cur[kStageWords];
+#pragma unroll
+                for (int i = 0; i < kStageWords; ++i) cur[i] = words[kStageWords * u + i];
+                const uint32_t s2 = sc_cur[u >> 1];  // one scale per 128 codes = two stages
+                uint32_t out[32];
+                if (row_ok) {
+                    expand_quads<0>(cur, s2, out);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) out[i] = 0u;
+                }
+                const int slot = s % kStages;
+                const uint32_t round = static_cast<uint32_t>(s / kStages);
+                ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar_empty + 8 * slot, (round & 1u) ^ 1u));
+                if (!ok) break;
+                if (t < p.tile_n) {
+                    const uint32_t row = b_base + slot * kBBytes + t * 128;
+#pragma unroll
+                    for (int jj = 0; jj < 8; ++jj) {
+                        const uint32_t dst = row + ((jj ^ (t & 7)) << 4);
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(out[4 * jj]),
+                                     "r"(out[4 * jj + 1]), "r"(out[4 * jj + 2]), "r"(out[4 * jj + 3])
+                                     : "memory");
+                    }
+                }
+                fence_async_smem();
+                mbar_arrive(bar_full_b + 8 * slot);
+            }
+            sc_cur[0] = sc_next[0];
+            sc_cur[1] = sc_next[1];
+        }
+#else
         // register ring: stage s lives in ring[s % kPrefetch]
         uint32_t ring[kPrefetch][kStageWords] = {};
         uint32_t ring_s[kPrefetch] = {};
@@ -306,6 +412,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                 mbar_arrive(bar_full_b + 8 * slot);
             }
         }
+
+#endif
 
         // ---- epilogue: TMEM -> bf16 -> y ----
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar_acc, 0));
