@@ -197,6 +197,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     const int n0 = blockIdx.x * p.tile_n;
     const int nstages = p.K / kStageK;
     const int G = p.K / kGroup;
+    // a batch tile of at most 128 rows needs only the first UMMA tile (mid-sized batches)
+    const bool two_tiles = m0 + kUmmaM < p.M;
     [[maybe_unused]] const int W = G * kWordsPerGroup;
 
     if (threadIdx.x == 0) {
@@ -231,10 +233,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                 const uint32_t round = static_cast<uint32_t>(s / kStages);
                 ok = mbar_wait_bounded(bar_empty + 8 * slot, (round & 1u) ^ 1u);
                 if (!ok) break;
-                mbar_arrive_expect_tx(bar_full_a + 8 * slot, 2 * kABytes);
+                mbar_arrive_expect_tx(bar_full_a + 8 * slot, (two_tiles ? 2 : 1) * kABytes);
                 const uint32_t dst = a_base + slot * 2 * kABytes;
                 tma_load_2d(dst, &p.tmap_x, s * kStageK, m0, bar_full_a + 8 * slot);
-                tma_load_2d(dst + kABytes, &p.tmap_x, s * kStageK, m0 + kUmmaM, bar_full_a + 8 * slot);
+                if (two_tiles) tma_load_2d(dst + kABytes, &p.tmap_x, s * kStageK, m0 + kUmmaM, bar_full_a + 8 * slot);
             }
         }
     } else if (warp == 1) {
@@ -255,7 +257,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
                 const uint64_t bd = desc_add(bd0, kk * 32);
                 const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
                 umma_bf16(tmem, desc_add(ad, kk * 32), bd, p.idesc, acc);
-                umma_bf16(d1, desc_add(ad, kABytes + kk * 32), bd, p.idesc, acc);
+                if (two_tiles) umma_bf16(d1, desc_add(ad, kABytes + kk * 32), bd, p.idesc, acc);
             }
             umma_commit(bar_empty + 8 * slot);  // frees the stage once these MMAs have read it
         }
@@ -424,7 +426,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             const int m = m0 + sub * kUmmaM + quarter * 32 + lane;
             const uint32_t tbase = tmem + (static_cast<uint32_t>(quarter * 32) << 16) +
                                    static_cast<uint32_t>(sub * p.tile_n);
-            for (int c0 = 0; c0 < p.tile_n; c0 += 32) {
+            const int cols = (sub == 0 || two_tiles) ? p.tile_n : 0;  // tile 1 holds nothing when unused
+            for (int c0 = 0; c0 < cols; c0 += 32) {
                 uint32_t v[32];
                 tmem_ld32(tbase + c0, v);
                 if (m < p.M) {
