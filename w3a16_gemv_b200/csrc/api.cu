@@ -299,13 +299,10 @@ w3_status launch_prefill(const uint16_t *x, const int32_t *packed, const uint16_
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return W3_ERR_CUDA;
-    if (W3_PREFILL_WTMA) {
-        // [BN rows][24 words] boxes over the packed matrix: four stages of the CTA's rows per copy
-        if (encode_packed_map(&prm.tmap_w, packed, N, static_cast<int64_t>(K) * 3 / 32,
-                              prefill::kChunkStages * prefill::kStageWords, static_cast<uint32_t>(P.tile_n)) != W3_OK)
-            return W3_ERR_CUDA;
-    }
-    prm.packed = reinterpret_cast<const uint32_t *>(packed);
+    // [BN rows][24 words] boxes over the packed matrix: four stages of the CTA's rows per copy
+    if (encode_packed_map(&prm.tmap_w, packed, N, static_cast<int64_t>(K) * 3 / 32,
+                          prefill::kChunkStages * prefill::kStageWords, static_cast<uint32_t>(P.tile_n)) != W3_OK)
+        return W3_ERR_CUDA;
     prm.scales = scales;
     prm.y = y;
     prm.M = M;

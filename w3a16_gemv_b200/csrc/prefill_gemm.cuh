@@ -12,19 +12,21 @@
 //    2 x BN columns of the 512 the CTA allocates.
 //  * A (x): one tiled TMA copy per 128-row tile and stage, 128-byte swizzle,
 //    the canonical K-major layout the UMMA descriptors describe.
-//  * B (W): 8 dequantizing warps, one W row per thread.  A stage of a row is
-//    64 codes = 6 packed words, loaded kPrefetch stages ahead into a register
-//    ring so that the global-load latency hides behind the expansions.  Codes are expanded
-//    in natural k order four at a time: the 12 bits of two code pairs times
-//    0x2001 place each pair's second code 13 bits above its first, so one
-//    LOP3 (mask | bf16 128.0) per pair gives (128 + c_k, 128 + c_k+1) exactly;
-//    a bf16x2 subtract of 132 gives the levels q = c - 4, and a bf16x2
-//    multiply by the group scale gives bf16(q * s), rounded once.  The row is
-//    stored into the stage's B buffer in the same 128-byte-swizzled K-major
-//    layout, then made visible to the tensor cores' async proxy.
-//  * One thread issues tcgen05.mma (kind::f16, bf16 x bf16 -> fp32) for both
-//    128-row tiles and commits each stage back to the producers.
-//  * Epilogue: the 8 warps read the accumulators with tcgen05.ld, round to
+//  * Packed W: one producer warp copies the CTA's rows, 24 words (four stages)
+//    per row and copy, into shared memory by TMA.
+//  * B (W): 8 dequantizing warps, one thread per W row (16 warps, two threads
+//    per row each expanding half of the row's 64 codes per stage, was slower).  Codes are expanded in natural k order
+//    four at a time: the 12 bits of two code pairs times 0x2001 place each
+//    pair's second code 13 bits above its first, so one LOP3 (mask | bf16
+//    128.0) per pair gives (128 + c_k, 128 + c_k+1) exactly; a bf16x2 subtract
+//    of 132 gives the levels q = c - 4, and a bf16x2 multiply by the group
+//    scale gives bf16(q * s), rounded once.  The halves are stored into the
+//    stage's B buffer in the 128-byte-swizzled K-major layout, then made
+//    visible to the tensor cores' async proxy.
+//  * One elected lane issues tcgen05.mma (kind::f16, bf16 x bf16 -> fp32) for
+//    both 128-row tiles (only the first when the batch tile holds <= 128 rows)
+//    and commits each stage back to the producers.
+//  * Epilogue: the dequantizing warps read the accumulators with tcgen05.ld, round to
 //    bf16 and store y.
 // All waits are bounded; a timeout is recorded and the CTA winds down.
 #pragma once
@@ -39,31 +41,23 @@ constexpr int kUmmaM = 128;
 constexpr int kMaxTileN = 256;       // rows of W per CTA at most
 constexpr int kStageK = 64;          // k per pipeline stage = one 128-byte swizzle atom of bf16
 constexpr int kStages = 3;
-constexpr int kDequantWarps = 8;     // one W row per thread: BN <= 256
-// 1: the packed words reach shared memory by TMA ([BN rows][24 words], four
-// stages per copy, from a producer warp) and each thread copies its row into
-// registers; 0: each thread loads its row's words from global memory.
-#ifndef W3_PREFILL_WTMA
-#define W3_PREFILL_WTMA 1
-#endif
-constexpr int kChunkStages = 4;                   // stages per packed-word copy
-constexpr int kThreads = (2 + kDequantWarps + (W3_PREFILL_WTMA ? 1 : 0)) * 32;
+constexpr int kDequantWarps = 8;     // 8: one thread per W row, 16: two (BN <= 256)
+constexpr int kHalves = 16 / kDequantWarps;  // 32-code halves of a stage per thread
+constexpr int kChunkStages = 4;      // stages per packed-word copy (an even number: whole groups)
+constexpr int kChunkGroups = kChunkStages / 2;
+constexpr int kThreads = (2 + kDequantWarps + 1) * 32;  // x TMA, MMA, dequant warps, packed-word TMA
 constexpr int kTmemCols = 512;
 constexpr int kABytes = kUmmaM * kStageK * 2;     // 16 KB per 128-row tile and stage
 constexpr int kBBytes = kMaxTileN * kStageK * 2;  // 32 KB per stage (BN rows used)
 constexpr int kStageWords = kStageK * 3 / 32;     // 6 packed words per row and stage
-#ifndef W3_PREFILL_PREFETCH
-#define W3_PREFILL_PREFETCH 4
-#endif
-constexpr int kPrefetch = W3_PREFILL_PREFETCH;      // stages of packed words in flight per thread
 
 struct SmemLayout {
     // all operand buffers are 1024-byte aligned (the 128-byte swizzle period)
     static constexpr int a_off = 0;                                  // [kStages][2][kABytes]
     static constexpr int b_off = a_off + kStages * 2 * kABytes;      // [kStages][kBBytes]
-    static constexpr int w_off = b_off + kStages * kBBytes;          // [BN rows][24 words] packed
-    static constexpr int sink_off = w_off + kMaxTileN * kChunkStages * 6 * 4;  // u32 [256]: see the release below
-    static constexpr int bar_off = sink_off + kMaxTileN * 4;         // full_a, full_b, empty [kStages], acc, w_full, w_empty
+    static constexpr int w_off = b_off + kStages * kBBytes;          // [BN rows][6 * kChunkStages words] packed
+    static constexpr int sink_off = w_off + kMaxTileN * kChunkStages * 6 * 4;  // u32 per dequant thread: see the release below
+    static constexpr int bar_off = sink_off + kDequantWarps * 32 * 4;  // full_a, full_b, empty [kStages], acc, w_full, w_empty
     static constexpr int tmem_slot_off = bar_off + (3 * kStages + 3) * 8;
     static constexpr int total = tmem_slot_off + 16 + 1024;          // + slack to align the base to 1024
 };
@@ -71,7 +65,6 @@ struct SmemLayout {
 struct Params {
     CUtensorMap tmap_x;  // x [M][K] bf16, box [128 rows][64 k], 128-byte swizzle
     CUtensorMap tmap_w;  // packed [N][3K/32] u32, box [BN rows][24 words]
-    const uint32_t *packed;
     const uint16_t *scales;
     uint16_t *y;
     int M, N, K;
@@ -148,14 +141,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-// Bits [12q, 12q+12) of the 192-bit stage stream w[0..5]: codes 4q..4q+3.
-template <int Q>
-__device__ __forceinline__ uint32_t quad_bits(const uint32_t (&w)[kStageWords]) {
-    constexpr int b = 12 * Q, i = b / 32, s = b % 32;
-    if constexpr (s + 12 <= 32) return (w[i] >> s) & 0xFFFu;
-    else return __funnelshift_r(w[i], w[i + 1], s) & 0xFFFu;
-}
-
 __device__ __forceinline__ uint32_t bf16x2_sub_mul(uint32_t v, uint32_t sub, uint32_t mul) {
     uint32_t q, r;
     asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(q) : "r"(v), "r"(sub));  // exact: c - 4
@@ -163,16 +148,20 @@ __device__ __forceinline__ uint32_t bf16x2_sub_mul(uint32_t v, uint32_t sub, uin
     return r;
 }
 
-// Expand one row's stage (64 codes) into 32 bf16x2 words of bf16(q*s), natural k order.
-template <int Q>
-__device__ __forceinline__ void expand_quads(const uint32_t (&w)[kStageWords], uint32_t s2, uint32_t (&out)[32]) {
-    if constexpr (Q < 16) {
-        constexpr uint32_t kMagic2 = 0x43004300u;  // bf16x2 (128, 128)
-        constexpr uint32_t kSub = 0x43044304u;     // bf16x2 (132, 132)
-        const uint32_t x = quad_bits<Q>(w) * 0x2001u;  // second code of each pair 13 bits above the first
-        out[2 * Q] = bf16x2_sub_mul(and_or<0x00070007u>(x, kMagic2), kSub, s2);
-        out[2 * Q + 1] = bf16x2_sub_mul(and_or<0x00070007u>(x >> 6, kMagic2), kSub, s2);
-        expand_quads<Q + 1>(w, s2, out);
+// Expand codes 4I .. 31 of a 96-bit half stage w[0..2] (32 codes) into bf16x2
+// words out[2I ..] of bf16(q*s), natural k order.
+template <int I>
+__device__ __forceinline__ void expand_half(const uint32_t (&w)[3], uint32_t s2, uint32_t magic, uint32_t sub,
+                                            uint32_t (&out)[16]) {
+    if constexpr (I < 8) {
+        constexpr int b = 12 * I, i = b / 32, sh = b % 32;
+        uint32_t bits;
+        if constexpr (sh + 12 <= 32) bits = (w[i] >> sh) & 0xFFFu;
+        else bits = __funnelshift_r(w[i], w[i + 1], sh) & 0xFFFu;
+        const uint32_t x = bits * 0x2001u;  // second code of each pair 13 bits above the first
+        out[2 * I] = bf16x2_sub_mul(and_or<0x00070007u>(x, magic), sub, s2);
+        out[2 * I + 1] = bf16x2_sub_mul(and_or<0x00070007u>(x >> 6, magic), sub, s2);
+        expand_half<I + 1>(w, s2, magic, sub, out);
     }
 }
 
@@ -188,28 +177,30 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     const uint32_t bar_empty = bar_full_b + 8 * kStages;
     const uint32_t bar_acc = bar_empty + 8 * kStages;
     const uint32_t bar_wfull = bar_acc + 8, bar_wempty = bar_acc + 16;
-    constexpr int kChunkWords = kChunkStages * kStageWords;  // 24 words per row and copy
+    constexpr int kChunkWords = kChunkStages * kStageWords;  // words per row and copy
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + SmemLayout::tmem_slot_off);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int m0 = blockIdx.y * kTileM;
-    const int n0 = blockIdx.x * p.tile_n;
+    // CTAs that share a W tile are adjacent in launch order, so they run together and the
+    // tile's packed words come from DRAM once and from L2 for the other batch tiles
+    const int mtiles = (p.M + kTileM - 1) / kTileM;
+    const int m0 = static_cast<int>(blockIdx.x % mtiles) * kTileM;
+    const int n0 = static_cast<int>(blockIdx.x / mtiles) * p.tile_n;
     const int nstages = p.K / kStageK;
     const int G = p.K / kGroup;
     // a batch tile of at most 128 rows needs only the first UMMA tile (mid-sized batches)
     const bool two_tiles = m0 + kUmmaM < p.M;
-    [[maybe_unused]] const int W = G * kWordsPerGroup;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(bar_full_a + 8 * s, 1);
-            mbar_init(bar_full_b + 8 * s, kDequantWarps * 32);
+            mbar_init(bar_full_b + 8 * s, kDequantWarps);  // one arrival per dequant warp
             mbar_init(bar_empty + 8 * s, 1);
         }
         mbar_init(bar_acc, 1);
         mbar_init(bar_wfull, 1);
-        mbar_init(bar_wempty, kDequantWarps * 32);
+        mbar_init(bar_wempty, kDequantWarps);
         mbar_init_fence();
     }
     if (warp == 1) {  // allocate the accumulators
@@ -274,24 +265,25 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             }
         }
     } else {
-        // ---- B producers: dequantize one W row per thread ----
-        const int t = threadIdx.x - 64;  // 0..255
-        const int n = n0 + t;
-        const bool row_ok = (t < p.tile_n) && (n < p.N);
-#if !W3_PREFILL_WTMA
-        const uint32_t *prow = p.packed + static_cast<int64_t>(row_ok ? n : 0) * W;
-#endif
+        // ---- B producers: row r of the tile; with 16 warps, half dw/8 of each stage's 64 codes ----
+        const int dw = warp - 2;             // 0 .. kDequantWarps-1
+        const int hsel = dw >> 3;            // the half this thread expands when kHalves == 1
+        const int r = (dw & 7) * 32 + lane;  // row of the tile
+        const int n = n0 + r;
+        const bool row_ok = (r < p.tile_n) && (n < p.N);
         const uint16_t *srow = p.scales + static_cast<int64_t>(row_ok ? n : 0) * G;
-#if W3_PREFILL_WTMA
+        const uint32_t *wsm = reinterpret_cast<const uint32_t *>(smem + SmemLayout::w_off);
+        uint32_t magic, sub;  // expansion constants, created once (opaque: not rebuilt before each use)
+        asm volatile("mov.b32 %0, %1;" : "=r"(magic) : "n"(0x43004300u));  // bf16x2 (128, 128)
+        asm volatile("mov.b32 %0, %1;" : "=r"(sub) : "n"(0x43044304u));    // bf16x2 (132, 132)
         // the row's 24 words of a 4-stage chunk come from the shared-memory copy; the chunk's two
         // group scales are loaded one chunk ahead
-        const uint32_t *wsm = reinterpret_cast<const uint32_t *>(smem + SmemLayout::w_off);
         const int nchunks = (nstages + kChunkStages - 1) / kChunkStages;
-        uint32_t sc_cur[2] = {0u, 0u}, sc_next[2] = {0u, 0u};
-        auto load_scales = [&](int c, uint32_t (&dst)[2]) {
+        uint32_t sc_cur[kChunkGroups] = {}, sc_next[kChunkGroups] = {};
+        auto load_scales = [&](int c, uint32_t (&dst)[kChunkGroups]) {
 #pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                const int g = 2 * c + i;
+            for (int i = 0; i < kChunkGroups; ++i) {
+                const int g = kChunkGroups * c + i;
                 const uint32_t hs = (row_ok && g < G) ? __ldg(srow + g) : 0u;
                 dst[i] = hs | (hs << 16);
             }
@@ -302,8 +294,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
             ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar_wfull, c & 1));
             if (!ok) break;
             uint32_t words[kChunkWords];
-            if (t < p.tile_n) {
-                const uint4 *src = reinterpret_cast<const uint4 *>(wsm + t * kChunkWords);
+            if (r < p.tile_n) {
+                const uint4 *src = reinterpret_cast<const uint4 *>(wsm + r * kChunkWords);
 #pragma unroll
                 for (int i = 0; i < kChunkWords / 4; ++i) {
                     const uint4 q = src[i];
@@ -316,118 +308,72 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
 #pragma unroll
                 for (int i = 0; i < kChunkWords; ++i) words[i] = 0u;
             }
-            // The next copy into the buffer is an async-proxy write, and the arrive below orders
-            // memory operations, not the arrival of load results in registers.  A store that
-            // depends on every loaded register therefore precedes the arrive: the buffer is
-            // released only once the loads have completed.
+            // The next copy into the buffer is an async-proxy write, and an arrive orders memory
+            // operations, not the arrival of load results in registers.  A store that depends on
+            // every loaded register therefore precedes the warp's arrival: the buffer is released
+            // only once every lane's loads have completed.
             uint32_t landed = 0;
 #pragma unroll
             for (int i = 0; i < kChunkWords; i += 4) landed ^= words[i];
-            asm volatile("st.shared.u32 [%0], %1;" ::"r"(sbase + SmemLayout::sink_off + 4 * t), "r"(landed) : "memory");
-            mbar_arrive(bar_wempty);
+            asm volatile("st.shared.u32 [%0], %1;" ::"r"(sbase + SmemLayout::sink_off + 4 * (threadIdx.x - 64)),
+                         "r"(landed)
+                         : "memory");
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_wempty);
 #pragma unroll
             for (int u = 0; u < kChunkStages; ++u) {
                 const int s = c * kChunkStages + u;
                 if (s >= nstages || !ok) break;
-                uint32_t cur[kStageWords];
-#pragma unroll
-                for (int i = 0; i < kStageWords; ++i) cur[i] = words[kStageWords * u + i];
                 const uint32_t s2 = sc_cur[u >> 1];  // one scale per 128 codes = two stages
-                uint32_t out[32];
-                if (row_ok) {
-                    expand_quads<0>(cur, s2, out);
-                } else {
+                uint32_t out[kHalves][16];
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) out[i] = 0u;
+                for (int hh = 0; hh < kHalves; ++hh) {
+                    uint32_t cur[3];  // half h of the stage: words 3h .. 3h+2
+#pragma unroll
+                    for (int i = 0; i < 3; ++i)
+                        cur[i] = (kHalves == 2) ? words[kStageWords * u + 3 * hh + i]
+                                                : (hsel ? words[kStageWords * u + 3 + i] : words[kStageWords * u + i]);
+                    expand_half<0>(cur, s2, magic, sub, out[hh]);
                 }
                 const int slot = s % kStages;
                 const uint32_t round = static_cast<uint32_t>(s / kStages);
                 ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar_empty + 8 * slot, (round & 1u) ^ 1u));
                 if (!ok) break;
-                if (t < p.tile_n) {
-                    const uint32_t row = b_base + slot * kBBytes + t * 128;
+                if (r < p.tile_n) {
+                    const uint32_t row = b_base + slot * kBBytes + r * 128;
 #pragma unroll
-                    for (int jj = 0; jj < 8; ++jj) {
-                        const uint32_t dst = row + ((jj ^ (t & 7)) << 4);
-                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(out[4 * jj]),
-                                     "r"(out[4 * jj + 1]), "r"(out[4 * jj + 2]), "r"(out[4 * jj + 3])
-                                     : "memory");
+                    for (int hh = 0; hh < kHalves; ++hh) {
+                        const int h = (kHalves == 2) ? hh : hsel;
+#pragma unroll
+                        for (int jj = 0; jj < 4; ++jj) {
+                            const uint32_t dst = row + (((4 * h + jj) ^ (r & 7)) << 4);
+                            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst),
+                                         "r"(out[hh][4 * jj]), "r"(out[hh][4 * jj + 1]), "r"(out[hh][4 * jj + 2]),
+                                         "r"(out[hh][4 * jj + 3])
+                                         : "memory");
+                        }
                     }
                 }
                 fence_async_smem();
-                mbar_arrive(bar_full_b + 8 * slot);
+                __syncwarp();  // the warp's stores are ordered before lane 0's arrival
+                if (lane == 0) mbar_arrive(bar_full_b + 8 * slot);
             }
-            sc_cur[0] = sc_next[0];
-            sc_cur[1] = sc_next[1];
-        }
-#else
-        // register ring: stage s lives in ring[s % kPrefetch]
-        uint32_t ring[kPrefetch][kStageWords] = {};
-        uint32_t ring_s[kPrefetch] = {};
-        auto load = [&](int s, uint32_t (&dst)[kStageWords], uint32_t &sc) {
-            if (row_ok && s < nstages) {
-                const uint2 *src = reinterpret_cast<const uint2 *>(prow + s * kStageWords);
 #pragma unroll
-                for (int i = 0; i < 3; ++i) {
-                    const uint2 v = __ldg(src + i);
-                    dst[2 * i] = v.x;
-                    dst[2 * i + 1] = v.y;
-                }
-                const uint32_t h = __ldg(srow + s / 2);  // one scale per 128 = two stages
-                sc = h | (h << 16);
-            }
-        };
-#pragma unroll
-        for (int u = 0; u < kPrefetch; ++u) load(u, ring[u], ring_s[u]);
-        for (int s0 = 0; s0 < nstages && ok; s0 += kPrefetch) {
-#pragma unroll
-            for (int u = 0; u < kPrefetch; ++u) {
-                const int s = s0 + u;
-                if (s >= nstages || !ok) break;
-                uint32_t cur[kStageWords];
-#pragma unroll
-                for (int i = 0; i < kStageWords; ++i) cur[i] = ring[u][i];
-                const uint32_t s2 = ring_s[u];
-                load(s + kPrefetch, ring[u], ring_s[u]);  // refill this ring slot
-                uint32_t out[32];
-                if (row_ok) {
-                    expand_quads<0>(cur, s2, out);
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) out[i] = 0u;
-                }
-                const int slot = s % kStages;
-                const uint32_t round = static_cast<uint32_t>(s / kStages);
-                ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar_empty + 8 * slot, (round & 1u) ^ 1u));
-                if (!ok) break;
-                if (t < p.tile_n) {
-                    const uint32_t row = b_base + slot * kBBytes + t * 128;
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const uint32_t dst = row + ((j ^ (t & 7)) << 4);
-                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(out[4 * j]),
-                                     "r"(out[4 * j + 1]), "r"(out[4 * j + 2]), "r"(out[4 * j + 3])
-                                     : "memory");
-                    }
-                }
-                fence_async_smem();
-                mbar_arrive(bar_full_b + 8 * slot);
-            }
+            for (int i = 0; i < kChunkGroups; ++i) sc_cur[i] = sc_next[i];
         }
 
-#endif
-
-        // ---- epilogue: TMEM -> bf16 -> y ----
+        // ---- epilogue: TMEM -> bf16 -> y; per TMEM lane quarter, kDequantWarps/4 warps share the tiles ----
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar_acc, 0));
         tc_fence_after();
         if (ok) {
-            const int quarter = warp & 3;           // TMEM lanes 32*quarter .. +31
-            const int sub = (warp - 2) / 4;         // warps 2-5: tile 0, warps 6-9: tile 1
-            const int m = m0 + sub * kUmmaM + quarter * 32 + lane;
+            const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
+            const int tsub = (dw >> 2) & 1;  // accumulator tile
+            const int ch = dw >> 3;          // with 16 warps: every other 32-column chunk
+            const int m = m0 + tsub * kUmmaM + quarter * 32 + lane;
             const uint32_t tbase = tmem + (static_cast<uint32_t>(quarter * 32) << 16) +
-                                   static_cast<uint32_t>(sub * p.tile_n);
-            const int cols = (sub == 0 || two_tiles) ? p.tile_n : 0;  // tile 1 holds nothing when unused
-            for (int c0 = 0; c0 < cols; c0 += 32) {
+                                   static_cast<uint32_t>(tsub * p.tile_n);
+            const int cols = (tsub == 0 || two_tiles) ? p.tile_n : 0;  // tile 1 holds nothing when unused
+            for (int c0 = 32 * ch; c0 < cols; c0 += 32 * (kDequantWarps / 8)) {
                 uint32_t v[32];
                 tmem_ld32(tbase + c0, v);
                 if (m < p.M) {
@@ -484,7 +430,7 @@ inline LaunchPlan plan(int M, int N, int num_sms) {
     }
     if (N < 128) best = (N + 31) / 32 * 32;
     P.tile_n = best;
-    P.grid = dim3((N + best - 1) / best, mt, 1);
+    P.grid = dim3(mt * ((N + best - 1) / best), 1, 1);  // batch tile fastest
     return P;
 }
 
