@@ -30,9 +30,11 @@
 //    turns each into the exact level q = c - 4 (the ten FMA constants are
 //    pinned in registers).  The group's 64 words go to the thread's
 //    tensor-memory lane (two tcgen05.st): the A operand.
-//  * One thread issues 8 tcgen05.mma per group and tile (A from tensor memory,
-//    B = permuted x from shared memory) into a fresh per-group fp32
-//    accumulator of 16 columns (four buffers per tile).
+//  * One warp per tile, on different SM sub-partitions, issues 8 tcgen05.mma
+//    per group from an elected lane (A from tensor memory, B = permuted x from
+//    shared memory) into a fresh per-group fp32 accumulator of 16 columns (four
+//    buffers per tile).  The issue of these short MMAs shares its sub-partition
+//    with two row warps and is what paces the kernel, hence one warp per tile.
 //  * The row threads read each group's 16 results back two groups later
 //    (tcgen05.ld) and add s[n,g] * D to fp32 registers: the group scale is
 //    applied in fp32 and nothing is rounded before the bf16 store.
@@ -85,7 +87,8 @@ constexpr int kTmemCols = kTiles * kTileCols;                 // 512 or 256 (two
 static_assert(kTmemCols * kCtasPerSm <= 512, "tensor memory per SM");
 constexpr int kRowWarps = kTiles * 4;
 constexpr int kScaleWarp = 2 + kRowWarps;                     // warp 10
-constexpr int kThreads = (3 + kRowWarps) * 32;                // load, MMA, row warps, scale warp
+constexpr int kMmaWarp1 = 3 + kRowWarps;                      // warp 11: the MMAs of tile 1 (warp 1: tile 0)
+constexpr int kThreads = (4 + kRowWarps) * 32;                // load, MMA x 2, row warps, scale warp
 constexpr int kScaleSlotBytes = kStageGroups * kRows * 2;     // [3 groups][256 rows] bf16
 
 #ifndef W3_DECODE_TC_MIN_UNITS
@@ -105,8 +108,8 @@ struct SmemLayout {
     static constexpr int stage_off = 0;  // [kStages]{x: [3][2 boxes], packed}
     static constexpr int scale_off = stage_off + kStages * kStageBytes;  // [kStages][3][256] bf16
     static constexpr int bar_off = scale_off + kStages * kScaleSlotBytes;
-    // full, empty, bready [kStages]; a_full [kTiles][kABuf]; done [kDBuf] (the MMAs of a group, both tiles)
-    static constexpr int nbars = 3 * kStages + kTiles * kABuf + kDBuf;
+    // full, empty, bready [kStages]; a_full [kTiles][kABuf]; done [kTiles][kDBuf] (the MMAs of a group and tile)
+    static constexpr int nbars = 3 * kStages + kTiles * kABuf + kTiles * kDBuf;
     static constexpr int tmem_slot_off = bar_off + nbars * 8;
     static constexpr int total = tmem_slot_off + 16 + 1024;  // + slack for 1024-byte alignment
 };
@@ -313,7 +316,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_tc_kernel(const _
     const uint32_t bars = sbase + SmemLayout::bar_off;
     const uint32_t bar_full = bars, bar_empty = bars + 8 * kStages, bar_bready = bars + 16 * kStages;
     const uint32_t bar_afull = bars + 24 * kStages;                // [kTiles][kABuf]
-    const uint32_t bar_done = bar_afull + 8 * kTiles * kABuf;      // [kDBuf]
+    const uint32_t bar_done = bar_afull + 8 * kTiles * kABuf;      // [kTiles][kDBuf]
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + SmemLayout::tmem_slot_off);
 
     const int warp = threadIdx.x >> 5;
@@ -325,11 +328,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_tc_kernel(const _
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(bar_full + 8 * s, 1 + 32);  // the TMA bytes and the 32 lanes of the scale warp
-            mbar_init(bar_empty + 8 * s, kRows + 1);  // row threads read the words, the MMAs read x
+            mbar_init(bar_empty + 8 * s, kRows + kTiles);  // row threads read the words, each tile's MMAs read x
             mbar_init(bar_bready + 8 * s, 1);
         }
         for (int b = 0; b < kTiles * kABuf; ++b) mbar_init(bar_afull + 8 * b, kTileRows);
-        for (int b = 0; b < kDBuf; ++b) mbar_init(bar_done + 8 * b, 1);
+        for (int b = 0; b < kTiles * kDBuf; ++b) mbar_init(bar_done + 8 * b, 1);
         mbar_init_fence();
     }
     if (warp == 1) {
@@ -393,41 +396,46 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_tc_kernel(const _
             }
         }
         if (ok && stage > 0) prep(stage - 1, prev_ns);
-    } else if (warp == 1) {
-        // ---- MMA issue: per group and tile, 8 MMAs into a fresh accumulator; the
-        //      whole warp runs the loop and one elected lane issues ----
+    } else if (warp == 1 || warp == kMmaWarp1) {
+        // ---- MMA issue, one warp per tile (on different SM sub-partitions): per group, 8 MMAs
+        //      into a fresh accumulator; the whole warp runs the loop and one elected lane issues ----
+        const int tile = warp == 1 ? 0 : 1;
+        const uint32_t tt = tmem + tile * kTileCols;
+        const uint32_t afull = bar_afull + 8 * tile * kABuf, done = bar_done + 8 * tile * kDBuf;
+        const uint64_t xdesc0 = sw128_kmajor_desc(sbase + SmemLayout::stage_off);
         Walk walk(p);
         int64_t t;
-        int g0, len, stage = 0, j = 0;
-        const uint64_t xdesc0 = sw128_kmajor_desc(sbase + SmemLayout::stage_off);
+        int g0, len, slot = 0, ab = 0, db = 0;
+        uint32_t sph = 0, aph = 0;  // phases of the stage ring and of the A-buffer ring
         while (ok && walk.next(t, g0, len)) {
             for (int gs = 0; gs < len && ok; gs += kStageGroups) {
                 const int ns = min(kStageGroups, len - gs);
-                const int slot = stage % kStages;
-                ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar_bready + 8 * slot, (stage / kStages) & 1));
+                ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar_bready + 8 * slot, sph));
                 const uint64_t xd = desc_add(xdesc0, slot * kStageBytes);
-                for (int jj = 0; jj < ns && ok; ++jj, ++j) {
-                    const int ab = j % kABuf, db = j % kDBuf;
-                    for (int tile = 0; tile < kTiles && ok; ++tile) {
-                        ok = __all_sync(0xffffffffu,
-                                        mbar_wait_bounded(bar_afull + 8 * (tile * kABuf + ab), (j / kABuf) & 1));
-                        if (!ok) break;
-                        tc_fence_after();
-                        const uint32_t tt = tmem + tile * kTileCols;
-                        const uint32_t dcol = tt + kDCol0 + db * kBatch, acol = tt + ab * kACols;
-#pragma unroll
-                        for (int kk = 0; kk < 8; ++kk) {
-                            const uint64_t bd = desc_add(xd, jj * kXGroupBytes + (kk >> 2) * kXBox + (kk & 3) * 32);
-                            if (kk == 0) umma_ts<false>(dcol, acol, bd, p.idesc);
-                            else umma_ts<true>(dcol, acol + kk * 8, bd, p.idesc);
-                        }
-                    }
+                for (int jj = 0; jj < ns && ok; ++jj) {
+                    ok = __all_sync(0xffffffffu, mbar_wait_bounded(afull + 8 * ab, aph));
                     if (!ok) break;
-                    umma_commit(bar_done + 8 * db);  // both tiles: A read, D written
+                    tc_fence_after();
+                    const uint32_t dcol = tt + kDCol0 + db * kBatch, acol = tt + ab * kACols;
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint64_t bd = desc_add(xd, jj * kXGroupBytes + (kk >> 2) * kXBox + (kk & 3) * 32);
+                        if (kk == 0) umma_ts<false>(dcol, acol, bd, p.idesc);
+                        else umma_ts<true>(dcol, acol + kk * 8, bd, p.idesc);
+                    }
+                    umma_commit(done + 8 * db);  // this tile: A read, D written
+                    if (++ab == kABuf) {
+                        ab = 0;
+                        aph ^= 1u;
+                    }
+                    db = (db + 1) % kDBuf;
                 }
                 if (!ok) break;
                 umma_commit(bar_empty + 8 * slot);
-                ++stage;
+                if (++slot == kStages) {
+                    slot = 0;
+                    sph ^= 1u;
+                }
             }
         }
     } else if (warp == kScaleWarp) {
@@ -464,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_tc_kernel(const _
         const int quarter = warp & 3;  // a warp reaches TMEM lanes 32*(warp % 4) .. +31
         const int r = tile * kTileRows + quarter * 32 + lane;
         const uint32_t tt = tmem + tile * kTileCols + (static_cast<uint32_t>(quarter * 32) << 16);
-        const uint32_t afull = bar_afull + 8 * tile * kABuf, done = bar_done;
+        const uint32_t afull = bar_afull + 8 * tile * kABuf, done = bar_done + 8 * tile * kDBuf;
         float acc[kBatch];
         float s0 = 0.f, s1 = 0.f;  // scales of the (at most kLag = 2) groups awaiting read-back
         static_assert(kLag == 2, "the read-back queue below holds two groups");
