@@ -24,7 +24,7 @@
  *   - all array pointers are DEVICE pointers (cudaMalloc'd or torch CUDA
  *     tensors) on the current device; the caller owns every buffer.  The
  *     only device memory the library allocates is the scratch of w3a16_gemm
- *     (at most 32 KB per SM, for partial sums), taken from and returned to a
+ *     (at most 64 KB per SM, for partial sums), taken from and returned to a
  *     private stream-ordered pool on `stream` within the call, so calls on
  *     different streams never share it;
  *   - bf16 values are passed as their 16-bit patterns (uint16_t);
@@ -125,10 +125,11 @@ w3_status w3_dequant_f32(const int32_t *packed, const uint16_t *scales, float *w
  *   packed [N, 3K/32] int32, scales [N, K/128] bf16 (the format above)
  *   y      [M,N] bf16, row-major; every element is written
  * Arithmetic: fp32 accumulation; the result is rounded once to bf16 (nearest
- * even).  For M <= 16 the weight enters the products exactly (q and the
- * scale are applied in fp32; K may be split over several thread blocks, whose
- * fp32 partial sums are added in a fixed order); for M > 16 each weight is
- * first rounded to bf16(q*s) and fed to the tensor cores.  Repeated calls
+ * even).  For M <= 16, and for M <= 32 when N >= 256, the weight enters the
+ * products exactly (q and the scale are applied in fp32; K may be split over
+ * several thread blocks, whose fp32 partial sums are added in a fixed order);
+ * for larger M each weight is first rounded to bf16(q*s) and fed to the
+ * tensor cores.  Repeated calls
  * with the same arguments give bit-identical y (no floating-point atomics).
  * Errors: W3_ERR_NULL, W3_ERR_SHAPE (M, N < 1; K < 128 or K % 128 != 0;
  * M*K, N*K or M*N above 2^40), W3_ERR_ALIGN, W3_ERR_ALIAS (y overlaps x,
@@ -140,8 +141,8 @@ w3_status w3a16_gemm(const uint16_t *x, const int32_t *packed, const uint16_t *s
 /*
  * w3a16_gemm_noalloc -- the same product y = x * W^T as w3a16_gemm, with the
  * same arguments, checks, errors and results, that allocates nothing: the
- * tensor-core decode (5 <= M <= 16, N >= 256) keeps its fp32 partial sums in a
- * fixed scratch array inside the library (about 5 MB of device memory per
+ * tensor-core decode (5 <= M <= 32, N >= 256) keeps its fp32 partial sums in a
+ * fixed scratch array inside the library (about 10.5 MB of device memory per
  * device, sized for up to 160 SMs) instead of a stream-ordered allocation;
  * every other shape runs exactly as in w3a16_gemm.  The format paper has no
  * counterpart to this call; it is for callers that may not allocate.

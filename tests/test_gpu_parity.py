@@ -52,6 +52,11 @@ SMALL = [
     (513, 200, 384, "uniform8", "lognormal", "normal"),
     (32, 28672, 1024, "uniform8", "lognormal", "normal"),   # 128 tiles at once: packed-word buffer reuse
     (32, 448, 8192, "gsq_5level", "absnormal", "normal"),   # 32 packed-word copies per tile
+    # the 32-wide tensor-core decode (17 <= M <= 32, N >= 256)
+    (17, 256, 1152, "uniform8", "lognormal", "normal"),           # one row tile, K split over CTAs
+    (20, 1000, 4224, "gsq_5level", "absnormal", "normal_outliers"),
+    (24, 28672, 256, "uniform8", "lognormal", "normal"),          # many row tiles, two groups
+    (31, 300, 8192, "uniform8", "lognormal", "normal"),
 ]
 
 
@@ -115,6 +120,22 @@ def test_batch_rows_match_single_row_calls(orc):
         assert_within_bound(y1, ref[m:m + 1], tol[m:m + 1], f"row {m}")
         same += int(np.array_equal(y1[0], yb[m]))
     print(f"batch-invariance: {same}/16 rows bit-identical between M=1 and M=16")
+
+
+def test_position_probe_32_wide(orc):
+    # 32 batch rows, each a unit vector: every column of the 32-wide decode picks one weight
+    N, K = 300, 512
+    p = make_problem(32, N, K, seed=16)
+    _, codes, scales = device_problem(p)
+    packed = w3_pack(codes)
+    w = orc.dequant_f32(orc.pack(p.codes), p.scales_bf16, K)
+    for k0 in range(0, K, 32):
+        eye = np.zeros((32, K), dtype=np.float32)
+        eye[np.arange(32), k0 + np.arange(32)] = 1.0
+        x = torch.from_numpy(eye).to(torch.bfloat16).cuda()
+        y = oracle.bf16_to_f64(from_dev_bf16(w3a16_gemm(x, packed, scales)))
+        want = w[:, k0:k0 + 32].T.astype(np.float64)
+        assert np.all(np.abs(y - want) <= 2.0 ** -8 * np.abs(want) + 1e-30), k0
 
 
 def test_position_probe(orc):

@@ -19,6 +19,8 @@ CASES = [
     (16, 1024, 8192),   # k/v_proj shape: every tile shared by several CTAs
     (5, 300, 1152),     # ragged N, K of 9 groups
     (1, 4096, 4096),    # a shape that needs no scratch (falls through to the decode kernels)
+    (32, 28672, 8192),  # the 32-wide decode: twice the partial-sum scratch per CTA
+    (20, 1024, 8192),
 ]
 
 

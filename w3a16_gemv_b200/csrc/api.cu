@@ -14,6 +14,12 @@
 #include "common.cuh"
 #include "decode_gemv.cuh"
 #include "decode_streamk.cuh"
+// the tensor-core decode, once per batch width (16: M <= 16; 32: 17 <= M <= 32)
+#include "decode_tcgen05.cuh"
+#undef W3_TC_NS
+#undef W3_TC_BATCH
+#define W3_TC_NS decode_tc32
+#define W3_TC_BATCH 32
 #include "decode_tcgen05.cuh"
 #include "format_kernels.cuh"
 #include "prefill_gemm.cuh"
@@ -90,8 +96,7 @@ w3_status device_setup(int *num_sms, cudaMemPool_t *pool = nullptr) {
                 return;
             }
         }
-        if (cudaFuncSetAttribute(decode_tc::decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 decode_tc::SmemLayout::total) != cudaSuccess) {
+        if (decode_tc::Instance::set_smem() != cudaSuccess || decode_tc32::Instance::set_smem() != cudaSuccess) {
             st.status = W3_ERR_CUDA;
             return;
         }
@@ -218,28 +223,27 @@ w3_status launch_decode_sk(const uint16_t *x, const int32_t *packed, const uint1
     return e == cudaSuccess ? W3_OK : W3_ERR_CUDA;
 }
 
-// Tensor-core decode (tcgen05, weights as the MMA's M dimension), M <= 16.
+// Tensor-core decode (tcgen05, weights as the MMA's M dimension), M <= I::batch.
 // Shared tiles are finished by the fix-up kernel, launched behind it with
 // programmatic dependent launch; their fp32 partial sums live in `partial`
-// (decode_tc::plan(...).ws_floats floats, unused when that is 0).  Returns
+// (I::make_plan(...).ws_floats floats, unused when that is 0).  Returns
 // W3_ERR_UNSUPPORTED, without launching, for shapes it does not take (N < 256).
+template <class I>
 w3_status launch_decode_tc(const uint16_t *x, const int32_t *packed, const uint16_t *scales, uint16_t *y, int M,
-                           int N, int K, const decode_tc::LaunchPlan &P, float *partial, cudaStream_t stream) {
-    if (N < decode_tc::kRows || M > decode_tc::kBatch) return W3_ERR_UNSUPPORTED;
-    decode_tc::Params prm;
+                           int N, int K, const typename I::PlanT &P, float *partial, cudaStream_t stream) {
+    if (N < I::rows || M > I::batch) return W3_ERR_UNSUPPORTED;
+    typename I::ParamsT prm;
     const int64_t words = static_cast<int64_t>(K) * 3 / 32;
-    if (encode_packed_map(&prm.tmap_w1, packed, N, words, decode_tc::kPitch1, decode_tc::kRows) != W3_OK)
-        return W3_ERR_CUDA;
-    prm.has_w3 = words >= decode_tc::kPitch3;
+    if (encode_packed_map(&prm.tmap_w1, packed, N, words, I::pitch1, I::rows) != W3_OK) return W3_ERR_CUDA;
+    prm.has_w3 = words >= I::pitch3;
     prm.tmap_w3 = prm.tmap_w1;
-    if (prm.has_w3 &&
-        encode_packed_map(&prm.tmap_w3, packed, N, words, decode_tc::kPitch3, decode_tc::kRows) != W3_OK)
+    if (prm.has_w3 && encode_packed_map(&prm.tmap_w3, packed, N, words, I::pitch3, I::rows) != W3_OK)
         return W3_ERR_CUDA;
     PFN_cuTensorMapEncodeTiled enc = tensor_map_encoder();
     if (!enc) return W3_ERR_CUDA;
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
-    cuuint32_t box[2] = {64, decode_tc::kBatch};
+    cuuint32_t box[2] = {64, static_cast<cuuint32_t>(I::batch)};
     cuuint32_t estr[2] = {1, 1};
     if (enc(&prm.tmap_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t *>(x), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -254,19 +258,19 @@ w3_status launch_decode_tc(const uint16_t *x, const int32_t *packed, const uint1
     prm.G = K / kGroup;
     prm.P = P.P;
     prm.U = P.U;
-    prm.idesc = prefill::make_idesc(decode_tc::kTileRows, decode_tc::kBatch);
+    prm.idesc = prefill::make_idesc(I::tile_rows, I::batch);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(P.P, 1, 1);
-    cfg.blockDim = dim3(decode_tc::kThreads, 1, 1);
-    cfg.dynamicSmemBytes = decode_tc::SmemLayout::total;
+    cfg.blockDim = dim3(I::threads, 1, 1);
+    cfg.dynamicSmemBytes = I::smem_bytes;
     cfg.stream = stream;
     cudaLaunchAttribute mattr[1];
     set_pdl(mattr[0]);
     cfg.attrs = mattr;
     cfg.numAttrs = W3_DECODE_PDL ? 1 : 0;
-    if (cudaLaunchKernelEx(&cfg, decode_tc::decode_tc_kernel, prm) != cudaSuccess) return W3_ERR_CUDA;
+    if (I::launch(cfg, prm) != cudaSuccess) return W3_ERR_CUDA;
     if (P.P == 1) return W3_OK;
-    decode_tc::FixupParams fp;
+    typename I::FixupT fp;
     fp.partial = partial;
     fp.y = y;
     fp.M = M;
@@ -276,13 +280,13 @@ w3_status launch_decode_tc(const uint16_t *x, const int32_t *packed, const uint1
     fp.U = P.U;
     cudaLaunchConfig_t fcfg = {};
     fcfg.gridDim = dim3(P.P - 1, 1, 1);
-    fcfg.blockDim = dim3(decode_tc::kRows, 1, 1);
+    fcfg.blockDim = dim3(I::rows, 1, 1);
     fcfg.stream = stream;
     cudaLaunchAttribute attr[1];
     set_pdl(attr[0]);
     fcfg.attrs = attr;
     fcfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&fcfg, decode_tc::decode_tc_fixup_kernel, fp) == cudaSuccess ? W3_OK : W3_ERR_CUDA;
+    return I::launch_fixup(fcfg, fp) == cudaSuccess ? W3_OK : W3_ERR_CUDA;
 }
 
 w3_status launch_prefill(const uint16_t *x, const int32_t *packed, const uint16_t *scales, uint16_t *y, int M,
@@ -378,7 +382,7 @@ w3_status launch_decode(const uint16_t *x, const int32_t *packed, const uint16_t
 // kernel reads is written by the main kernel of the same call, so nothing in
 // it has to start at zero.
 constexpr int kNoAllocMaxCtas = 160 * decode_tc::kCtasPerSm;
-constexpr int64_t kNoAllocScratchFloats = int64_t(kNoAllocMaxCtas) * 2 * decode_tc::kBatch * decode_tc::kRows;
+constexpr int64_t kNoAllocScratchFloats = int64_t(kNoAllocMaxCtas) * 2 * decode_tc32::kBatch * decode_tc32::kRows;
 static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchFloats];
 
 struct NoAllocState {
@@ -504,6 +508,20 @@ w3_status w3a16_gemm(const uint16_t *x, const int32_t *packed, const uint16_t *s
     cudaMemPool_t pool;
     if (w3_status s = device_setup(&sms, &pool)) return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    // 17 <= M <= 32: the 32-wide tensor-core decode (N >= 256)
+    if (M > 16 && M <= decode_tc32::kBatch && N >= decode_tc32::kRows) {
+        const decode_tc32::LaunchPlan plan32 = decode_tc32::plan(N, K, sms);
+        float *partial = nullptr;
+        if (plan32.ws_floats > 0 &&
+            cudaMallocFromPoolAsync(reinterpret_cast<void **>(&partial), plan32.ws_floats * sizeof(float), pool, st) !=
+                cudaSuccess)
+            return W3_ERR_CUDA;
+        w3_status status = launch_decode_tc<decode_tc32::Instance>(x, packed, scales, y, static_cast<int>(M),
+                                                                   static_cast<int>(N), static_cast<int>(K), plan32,
+                                                                   partial, st);
+        if (partial && cudaFreeAsync(partial, st) != cudaSuccess && status == W3_OK) status = W3_ERR_CUDA;
+        return status;
+    }
     // the prefill kernel's packed-word copies are 24 words wide: rows of at least 256 codes
     if (M > 16 && W3_PREFILL_TCGEN05 && K >= 256)
         return launch_prefill(x, packed, scales, y, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), sms,
@@ -522,8 +540,8 @@ w3_status w3a16_gemm(const uint16_t *x, const int32_t *packed, const uint16_t *s
     for (int64_t m0 = 0; m0 < M && status == W3_OK; m0 += 16) {
         const int mb = static_cast<int>(std::min<int64_t>(16, M - m0));
         if (tc && mb >= W3_DECODE_TC_MIN_M) {
-            status = launch_decode_tc(x + m0 * K, packed, scales, y + m0 * N, mb, static_cast<int>(N),
-                                      static_cast<int>(K), tplan, partial, st);
+            status = launch_decode_tc<decode_tc::Instance>(x + m0 * K, packed, scales, y + m0 * N, mb,
+                                                           static_cast<int>(N), static_cast<int>(K), tplan, partial, st);
             if (status == W3_OK) continue;
             if (status != W3_ERR_UNSUPPORTED) break;
             status = W3_OK;
@@ -550,15 +568,23 @@ w3_status w3a16_gemm_noalloc(const uint16_t *x, const int32_t *packed, const uin
         return W3_ERR_ALIAS;
     int sms;
     if (w3_status s = device_setup(&sms)) return s;
-    // Only the tensor-core decode (W3_DECODE_TC_MIN_M <= M <= 16, N >= 256) uses
+    // Only the tensor-core decode (W3_DECODE_TC_MIN_M <= M <= 32, N >= 256) uses
     // scratch; every other shape takes w3a16_gemm's path, which allocates nothing.
-    if (M > 16 || M < W3_DECODE_TC_MIN_M || N < decode_tc::kRows) return w3a16_gemm(x, packed, scales, y, M, N, K, stream);
-    const decode_tc::LaunchPlan tplan = decode_tc::plan(N, K, sms);
-    if (tplan.ws_floats > kNoAllocScratchFloats) return W3_ERR_UNSUPPORTED;
+    if (M > decode_tc32::kBatch || M < W3_DECODE_TC_MIN_M || N < decode_tc::kRows)
+        return w3a16_gemm(x, packed, scales, y, M, N, K, stream);
     float *scratch = noalloc_scratch();
     if (!scratch) return W3_ERR_CUDA;
-    return launch_decode_tc(x, packed, scales, y, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K),
-                            tplan, scratch, reinterpret_cast<cudaStream_t>(stream));
+    const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (M > decode_tc::kBatch) {
+        const decode_tc32::LaunchPlan plan32 = decode_tc32::plan(N, K, sms);
+        if (plan32.ws_floats > kNoAllocScratchFloats) return W3_ERR_UNSUPPORTED;
+        return launch_decode_tc<decode_tc32::Instance>(x, packed, scales, y, static_cast<int>(M), static_cast<int>(N),
+                                                       static_cast<int>(K), plan32, scratch, st);
+    }
+    const decode_tc::LaunchPlan tplan = decode_tc::plan(N, K, sms);
+    if (tplan.ws_floats > kNoAllocScratchFloats) return W3_ERR_UNSUPPORTED;
+    return launch_decode_tc<decode_tc::Instance>(x, packed, scales, y, static_cast<int>(M), static_cast<int>(N),
+                                                 static_cast<int>(K), tplan, scratch, st);
 }
 
 w3_status w3_check_device_error(w3_stream_t stream) {

@@ -38,14 +38,22 @@
 //  * The row threads read each group's 16 results back two groups later
 //    (tcgen05.ld) and add s[n,g] * D to fp32 registers: the group scale is
 //    applied in fp32 and nothing is rounded before the bf16 store.
-#pragma once
+// The file is compiled once per batch width, in its own namespace: W3_TC_NS
+// names the instance and W3_TC_BATCH is its UMMA N, 16 (M <= 16) or 32
+// (17 <= M <= 32).  Without them it is the 16-wide instance, decode_tc.
+#ifndef W3_TC_NS
+#define W3_TC_NS decode_tc
+#endif
+#ifndef W3_TC_BATCH
+#define W3_TC_BATCH 16
+#endif
 
 #include "common.cuh"
 #include "decode_gemv.cuh"
 #include "prefill_gemm.cuh"
 
 namespace w3 {
-namespace decode_tc {
+namespace W3_TC_NS {
 
 using decode::pair_spec;
 using prefill::desc_add;
@@ -59,7 +67,8 @@ using prefill::umma_commit;
 constexpr int kTileRows = 128;                    // UMMA M: one tensor-memory lane per row
 constexpr int kTiles = 2;                         // row tiles per CTA, sharing x
 constexpr int kRows = kTiles * kTileRows;         // 256 rows per CTA (one TMA box)
-constexpr int kBatch = 16;                        // UMMA N
+constexpr int kBatch = W3_TC_BATCH;               // UMMA N
+static_assert(kBatch == 16 || kBatch == 32, "batch widths 16 and 32");
 constexpr int kStageGroups = 3;
 // Resident CTAs per SM and, with them, the per-CTA budgets of shared and
 // tensor memory: one CTA with 4 stages and 3 A buffers per tile, or two CTAs
@@ -69,15 +78,16 @@ constexpr int kStageGroups = 3;
 #endif
 constexpr int kCtasPerSm = W3_DECODE_TC_CTAS_PER_SM;
 static_assert(kCtasPerSm == 1 || kCtasPerSm == 2, "one or two CTAs per SM");
-constexpr int kStages = kCtasPerSm == 1 ? 4 : 2;
+static_assert(kBatch == 16 || kCtasPerSm == 1, "the 32-wide instance needs the one-CTA budget");
+constexpr int kStages = kBatch == 32 ? 3 : kCtasPerSm == 1 ? 4 : 2;
 constexpr int kPitch3 = kStageGroups * kWordsPerGroup;        // 36 words: rows of a 3-group box
 constexpr int kPitch1 = kWordsPerGroup;                       // 12 words: rows of a 1-group box
 constexpr int kBox1Bytes = kRows * kPitch1 * 4;               // 12 KB
-constexpr int kXBox = kBatch * 64 * 2;                        // 2 KB: [16 rows][64 k] bf16
+constexpr int kXBox = kBatch * 64 * 2;                        // 2 or 4 KB: [batch rows][64 k] bf16
 constexpr int kXGroupBytes = 2 * kXBox;                       // 4 KB
 constexpr int kXBytes = kStageGroups * kXGroupBytes;          // 12 KB
 constexpr int kStageBytes = kXBytes + kStageGroups * kBox1Bytes;  // 48 KB
-constexpr int kABuf = kCtasPerSm == 1 ? 3 : 1;                // A buffers (one group each) per tile
+constexpr int kABuf = kBatch == 32 ? 2 : kCtasPerSm == 1 ? 3 : 1;  // A buffers (one group each) per tile
 constexpr int kDBuf = 4;                                      // accumulators per tile
 constexpr int kLag = 2;                                       // groups between MMA and read-back
 constexpr int kACols = 64;                                    // 128 codes, two bf16 per column
@@ -240,6 +250,23 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// kBatch (16 or 32) consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld_batch(uint32_t taddr, uint32_t (&v)[kBatch]) {
+#if W3_TC_BATCH == 16
+    tmem_ld16(taddr, v);
+#else
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+          "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+          "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#endif
+}
+
 // Half H of a group's 128 codes (blocks 2H, 2H+1; 6 of the 12 words) as 32
 // bf16x2 words of exact levels in pair order: word 16*b + i holds codes
 // (lo_i, hi_i) of block 2H + b.
@@ -263,9 +290,9 @@ __device__ __forceinline__ void half_levels(const uint32_t (&w)[kWordsPerGroup],
 __device__ __forceinline__ void permute_x(uint8_t *xs, int ns, int lane) {
     for (int jj = 0; jj < ns; ++jj) {
 #pragma unroll
-        for (int it = 0; it < 2; ++it) {
-            const int item = lane + 32 * it;  // 16 rows x 4 blocks
-            const int r = item & 15, bl = item >> 4;
+        for (int it = 0; it < kBatch / 8; ++it) {
+            const int item = lane + 32 * it;  // kBatch rows x 4 blocks
+            const int r = item % kBatch, bl = item / kBatch;
             uint8_t *row = xs + jj * kXGroupBytes + (bl >> 1) * kXBox + r * 128;
             const int h = bl & 1, sw = r & 7;
             uint32_t src[16];
@@ -484,7 +511,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_tc_kernel(const _
             if (!ok) return;
             tc_fence_after();
             uint32_t v[kBatch];
-            tmem_ld16(tt + kDCol0 + db * kBatch, v);
+            tmem_ld_batch(tt + kDCol0 + db * kBatch, v);
 #pragma unroll
             for (int b = 0; b < kBatch; ++b) acc[b] = fmaf(sg, __uint_as_float(v[b]), acc[b]);
         };
@@ -635,5 +662,24 @@ inline LaunchPlan plan(int64_t N, int64_t K, int num_sms) {
     return L;
 }
 
-}  // namespace decode_tc
+// What the host launcher needs of this instance.
+struct Instance {
+    static constexpr int batch = kBatch, rows = kRows, tile_rows = kTileRows, threads = kThreads;
+    static constexpr int pitch1 = kPitch1, pitch3 = kPitch3, smem_bytes = SmemLayout::total;
+    using ParamsT = Params;
+    using FixupT = FixupParams;
+    using PlanT = LaunchPlan;
+    static PlanT make_plan(int64_t N, int64_t K, int sms) { return plan(N, K, sms); }
+    static cudaError_t set_smem() {
+        return cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SmemLayout::total);
+    }
+    static cudaError_t launch(const cudaLaunchConfig_t &cfg, const Params &prm) {
+        return cudaLaunchKernelEx(&cfg, decode_tc_kernel, prm);
+    }
+    static cudaError_t launch_fixup(const cudaLaunchConfig_t &cfg, const FixupParams &fp) {
+        return cudaLaunchKernelEx(&cfg, decode_tc_fixup_kernel, fp);
+    }
+};
+
+}  // namespace W3_TC_NS
 }  // namespace w3
