@@ -58,6 +58,13 @@ def kernel_name(M: int) -> str:
     return f"w3::decode_tc::decode_tc_kernel (M={M})"
 
 
+def kernels_per_call(M: int) -> int:
+    """Kernels w3a16_gemm launches for a decode batch of M rows on the gate_proj shape: the
+    tensor-core decode (M > 4) is followed by its partial-sum fix-up kernel (its work is split
+    over every SM, so some row tiles are shared)."""
+    return 1 if M <= 4 else 2
+
+
 def step_bytes() -> int:
     return sum(algorithmic_bytes(m, N_ROWS, K_COLS) for m in BATCHES)
 
@@ -578,9 +585,9 @@ def run_gpu(args):
     torch.cuda.synchronize()
     w3_check_device_error()
 
-    # ---- timed region: K steps, barrier + synchronize on both sides ----
-    events = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
-               for _ in BATCHES] for _ in range(args.steps)]
+    # ---- timed region: K steps back to back, barrier + synchronize on both sides.  Nothing is
+    #      recorded between the calls, so a call's kernel may start its set-up while the previous
+    #      one finishes (programmatic dependent launch), as in a model's decode step ----
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local)
     sampler.start()
@@ -591,7 +598,7 @@ def run_gpu(args):
     w0 = time.perf_counter()
     t_start.record(stream)
     for i in range(args.steps):
-        one_step(args.warmup + i, events[i])
+        one_step(args.warmup + i)
     t_end.record(stream)
     torch.cuda.synchronize()
     w1 = time.perf_counter()
@@ -600,7 +607,17 @@ def run_gpu(args):
     sampler.stop()
     w3_check_device_error()
     elapsed_ms = t_start.elapsed_time(t_end)
-    per_call_ms = {m: [events[i][j][0].elapsed_time(events[i][j][1]) for i in range(args.steps)]
+
+    # ---- per-call breakdown (second timed pass): an event pair around every call, which also
+    #      keeps consecutive calls from overlapping; the roofline's per-launch time comes from here ----
+    brk_steps = min(args.steps, 500)
+    events = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
+               for _ in BATCHES] for _ in range(brk_steps)]
+    for i in range(brk_steps):
+        one_step(args.warmup + args.steps + i, events[i])
+    torch.cuda.synchronize()
+    w3_check_device_error()
+    per_call_ms = {m: [events[i][j][0].elapsed_time(events[i][j][1]) for i in range(brk_steps)]
                    for j, m in enumerate(BATCHES)}
 
     if world > 1:
@@ -682,7 +699,9 @@ def run_gpu(args):
         "calls": calls,
         "roofline": roofline,
         "e2e": e2e,
-        "gpu_launches": args.steps * calls_per_step,
+        "gpu_launches": args.steps * sum(kernels_per_call(m) for m in BATCHES),
+        "per_call_timing": f"calls[]: CUDA events around each call over {brk_steps} further steps (no overlap "
+                           "between calls); value: the K steps back to back",
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
