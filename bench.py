@@ -172,6 +172,23 @@ def dist_setup():
     return world, rank, local
 
 
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The slowest rank's time: every rank's measurement all-reduced with MAX (a no-op for one rank).
+    Every rank must call it at the same point."""
+    if world <= 1:
+        return ms
+    import torch
+
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank: float, world: int, max_ms: float) -> float:
+    """Whole-job throughput per second: the units all replicas processed over the slowest rank's time."""
+    return units_per_rank * world / (max_ms * 1e-3)
+
+
 # --------------------------------------------------------------------------------------
 # CPU oracle (the reported baseline and the reference arm)
 # --------------------------------------------------------------------------------------
@@ -297,12 +314,9 @@ def run_prefill(args):
     w3_check_device_error()
     per_ms = [a.elapsed_time(b) for a, b in ev]
     total_ms = ev[0][0].elapsed_time(ev[-1][1])
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, world, dev)
     flop = 2.0 * M * N * K
-    value = flop * args.steps * world / (total_ms * 1e-3) / 1e12
+    value = job_throughput(flop * args.steps, world, total_ms) / 1e12
     # a timed region of a second or more runs the tensor cores under the power cap: compare with
     # the sustained figure; a short one with the burst figure
     peak, src = measured_tensor_peak(sustained=total_ms >= 1000.0)
@@ -620,13 +634,8 @@ def run_gpu(args):
     per_call_ms = {m: [events[i][j][0].elapsed_time(events[i][j][1]) for i in range(brk_steps)]
                    for j, m in enumerate(BATCHES)}
 
-    if world > 1:
-        t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
-
-    total_bytes = step_bytes() * args.steps * world
-    value = total_bytes / (elapsed_ms * 1e-3) / 1e9
+    elapsed_ms = max_over_ranks(elapsed_ms, world, dev)
+    value = job_throughput(step_bytes() * args.steps, world, elapsed_ms) / 1e9
     ms_per_step = elapsed_ms / args.steps
 
     # ---- roofline of the dominant kernel (largest share of the step) ----
@@ -675,11 +684,8 @@ def run_gpu(args):
     for i in range(e2e_steps):
         e2e_step(i)
     e_ms = (time.perf_counter() - e0) * 1e3
-    if world > 1:
-        t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e_ms = float(t.item())
-    e2e = {"value": step_bytes() * e2e_steps * world / (e_ms * 1e-3) / 1e9, "unit": UNIT,
+    e_ms = max_over_ranks(e_ms, world, dev)
+    e2e = {"value": job_throughput(step_bytes() * e2e_steps, world, e_ms) / 1e9, "unit": UNIT,
            "h2d_bytes_per_step": sum(m * K_COLS * 2 for m in BATCHES),
            "d2h_bytes_per_step": sum(m * N_ROWS * 2 for m in BATCHES),
            "steps": e2e_steps, "ms_per_step": e_ms / e2e_steps}
