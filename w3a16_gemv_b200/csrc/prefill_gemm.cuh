@@ -14,20 +14,23 @@
 //    the canonical K-major layout the UMMA descriptors describe.
 //  * Packed W: one producer warp copies the CTA's rows, 24 words (four stages)
 //    per row and copy, into shared memory by TMA.
-//  * B (W): 8 dequantizing warps, one thread per W row (16 warps, two threads
-//    per row each expanding half of the row's 64 codes per stage, was slower).  Codes are expanded in natural k order
-//    four at a time: the 12 bits of two code pairs times 0x2001 place each
-//    pair's second code 13 bits above its first, so one LOP3 (mask | bf16
-//    128.0) per pair gives (128 + c_k, 128 + c_k+1) exactly; a bf16x2 subtract
-//    of 132 gives the levels q = c - 4, and a bf16x2 multiply by the group
-//    scale gives bf16(q * s), rounded once.  The halves are stored into the
-//    stage's B buffer in the 128-byte-swizzled K-major layout, then made
-//    visible to the tensor cores' async proxy.
+//  * B (W): 8 dequantizing warps, one thread per W row (kDequantWarps = 16,
+//    two threads per row each expanding half of a stage's 64 codes, is built
+//    too and was slower).  Codes are expanded in natural k order four at a
+//    time: the 12 bits of two code pairs times 0x2001 place each pair's second
+//    code 13 bits above its first, so one LOP3 (mask | bf16 128.0) per pair
+//    gives (128 + c_k, 128 + c_k+1) exactly; a bf16x2 subtract of 132 gives the
+//    levels q = c - 4, and a bf16x2 multiply by the group scale gives
+//    bf16(q * s), rounded once.  The rows are stored into the stage's B buffer
+//    in the 128-byte-swizzled K-major layout, then made visible to the tensor
+//    cores' async proxy; one arrival per warp hands the stage over.
 //  * One elected lane issues tcgen05.mma (kind::f16, bf16 x bf16 -> fp32) for
 //    both 128-row tiles (only the first when the batch tile holds <= 128 rows)
 //    and commits each stage back to the producers.
-//  * Epilogue: the dequantizing warps read the accumulators with tcgen05.ld, round to
-//    bf16 and store y.
+//  * Launch order: the batch tile varies fastest, so the CTAs sharing a W tile
+//    run side by side and its packed words come from DRAM once.
+//  * Epilogue: the dequantizing warps read the accumulators with tcgen05.ld,
+//    round to bf16 and store y.
 // All waits are bounded; a timeout is recorded and the CTA winds down.
 #pragma once
 
