@@ -45,6 +45,12 @@ SMALL = [
     (13, 28672, 256, "uniform8", "lognormal", "normal"),          # many row tiles, two groups
     (1, 2000, 128, "uniform8", "lognormal", "normal"),
     (1, 64, 28672, "gsq_5level", "absnormal", "normal_outliers"),
+    # the stream-K decode (M <= 4 with at least as many 32-row blocks as SMs): ragged blocks,
+    # odd group counts, blocks split between warps
+    (1, 4800, 384, "uniform8", "lognormal", "normal"),
+    (3, 5000, 1152, "gsq_5level", "absnormal", "normal_outliers"),
+    (4, 6000, 640, "uniform8", "lognormal", "normal"),
+    (2, 4736, 3968, "gsq_uniform", "lognormal", "normal"),
     (17, 50, 512, "uniform8", "lognormal", "normal"),
     (40, 96, 1280, "uniform8", "lognormal", "normal"),
     (256, 256, 256, "uniform8", "lognormal", "normal"),

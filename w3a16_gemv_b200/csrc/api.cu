@@ -546,7 +546,9 @@ w3_status w3a16_gemm(const uint16_t *x, const int32_t *packed, const uint16_t *s
             if (status != W3_ERR_UNSUPPORTED) break;
             status = W3_OK;
         }
-        const bool sk = W3_DECODE_STREAMK && decode_sk::applicable(mb, static_cast<int>(N), static_cast<int>(K));
+        // fewer 32-row blocks than SMs: the cluster split-K decode spreads K over more SMs
+        const bool sk = W3_DECODE_STREAMK && N >= static_cast<int64_t>(decode_sk::kBlockRows) * sms &&
+                        decode_sk::applicable(mb, static_cast<int>(N), static_cast<int>(K));
         status = sk ? launch_decode_sk(x + m0 * K, packed, scales, y + m0 * N, mb, static_cast<int>(N),
                                        static_cast<int>(K), sms, st)
                     : launch_decode(x + m0 * K, packed, scales, y + m0 * N, mb, static_cast<int>(N),
