@@ -51,6 +51,10 @@ SMALL = [
     (3, 5000, 1152, "gsq_5level", "absnormal", "normal_outliers"),
     (4, 6000, 640, "uniform8", "lognormal", "normal"),
     (2, 4736, 3968, "gsq_uniform", "lognormal", "normal"),
+    # a single group (K = 128) on every path: tcgen05 decode 16 and 32 wide, 16-row passes above 32
+    (8, 512, 128, "uniform8", "lognormal", "normal"),
+    (24, 512, 128, "uniform8", "lognormal", "normal"),
+    (40, 300, 128, "gsq_5level", "absnormal", "normal"),
     (17, 50, 512, "uniform8", "lognormal", "normal"),
     (40, 96, 1280, "uniform8", "lognormal", "normal"),
     (256, 256, 256, "uniform8", "lognormal", "normal"),
