@@ -220,3 +220,8 @@ def test_full_size_sampled(orc, name):
 
 def test_prefill_full_size_sampled(orc):
     _sampled_check(orc, "prefill_2048x28672x8192", n_samples=4096)
+
+
+def test_prefill_tensor_memory_kernel_full_size_sampled(orc):
+    # M = 1024 on gate_proj: the weights-in-tensor-memory prefill kernel is the one launched
+    _sampled_check(orc, "prefill_1024x28672x8192", n_samples=4096)

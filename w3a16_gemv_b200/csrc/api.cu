@@ -4,6 +4,7 @@
 // launch.  All arithmetic runs in the kernels included below (one translation
 // unit, so the device error flag needs no relocatable device code).
 #include <atomic>
+#include <cmath>
 #include <cstdint>
 #include <mutex>
 
@@ -23,6 +24,7 @@
 #include "decode_tcgen05.cuh"
 #include "format_kernels.cuh"
 #include "prefill_gemm.cuh"
+#include "prefill_swab.cuh"
 
 #ifndef W3_DECODE_TMA2D
 #define W3_DECODE_TMA2D 1
@@ -37,6 +39,10 @@
 // Launch the decode kernels with programmatic dependent launch.
 #ifndef W3_DECODE_PDL
 #define W3_DECODE_PDL 1
+#endif
+// The prefill with the weights in tensor memory (prefill_swab.cuh): a candidate for M >= 256.
+#ifndef W3_PREFILL_SWAB
+#define W3_PREFILL_SWAB 1
 #endif
 #ifndef W3_DECODE_TC_MIN_M
 #define W3_DECODE_TC_MIN_M 5
@@ -107,6 +113,11 @@ w3_status device_setup(int *num_sms, cudaMemPool_t *pool = nullptr) {
         uint64_t keep = UINT64_MAX;
         if (cudaMemPoolCreate(&st.pool, &props) != cudaSuccess ||
             cudaMemPoolSetAttribute(st.pool, cudaMemPoolAttrReleaseThreshold, &keep) != cudaSuccess) {
+            st.status = W3_ERR_CUDA;
+            return;
+        }
+        if (cudaFuncSetAttribute(prefill_ab::prefill_ab_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 prefill_ab::SmemLayout::total) != cudaSuccess) {
             st.status = W3_ERR_CUDA;
             return;
         }
@@ -322,6 +333,58 @@ w3_status launch_prefill(const uint16_t *x, const int32_t *packed, const uint16_
     return cudaLaunchKernelEx(&cfg, prefill::prefill_kernel, prm) == cudaSuccess ? W3_OK : W3_ERR_CUDA;
 }
 
+// Which prefill kernel: both are paced by full waves of CTAs.  A wave of the shared-memory
+// kernel takes about 43 + 0.27 * BN us at K = 8192 (its dequantizing producers do not speed up
+// in proportion to a smaller tile), a wave of the tensor-memory kernel (256 x rows per tile)
+// about 55 us (measured on B200 over gate/down/q-shaped problems); the shared-memory kernel is
+// kept unless the other is predicted 2 % faster, and below 256 rows of x, where its CTA time
+// does not shrink with the batch.
+bool prefer_prefill_ab(int M, int N, int sms) {
+    if (M < prefill_ab::kMaxBN) return false;
+    const prefill::LaunchPlan po = prefill::plan(M, N, sms);
+    const prefill_ab::LaunchPlan pa = prefill_ab::plan(M, N);
+    const double waves_o = std::ceil(static_cast<double>(po.grid.x) * po.grid.y / sms);
+    const double waves_a = std::ceil(static_cast<double>(pa.grid.x) / sms);
+    const double cost_o = waves_o * (43.0 + 0.27 * po.tile_n);
+    const double cost_a = waves_a * 55.0;
+    return cost_a < 0.98 * cost_o;
+}
+
+// Prefill with the weights in tensor memory (prefill_swab.cuh).
+w3_status launch_prefill_ab(const uint16_t *x, const int32_t *packed, const uint16_t *scales, uint16_t *y, int M,
+                            int N, int K, cudaStream_t stream) {
+    const prefill_ab::LaunchPlan P = prefill_ab::plan(M, N);
+    prefill_ab::Params prm;
+    PFN_cuTensorMapEncodeTiled enc = tensor_map_encoder();
+    if (!enc) return W3_ERR_CUDA;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+    cuuint32_t box[2] = {prefill_ab::kStageK, static_cast<cuuint32_t>(P.bn)};
+    cuuint32_t estr[2] = {1, 1};
+    if (enc(&prm.tmap_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t *>(x), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return W3_ERR_CUDA;
+    // [128 rows][24 words] boxes over the packed matrix: four stages of the CTA's rows per copy
+    if (encode_packed_map(&prm.tmap_w, packed, N, static_cast<int64_t>(K) * 3 / 32, prefill_ab::kChunkWords,
+                          prefill_ab::kRowsW) != W3_OK)
+        return W3_ERR_CUDA;
+    prm.scales = scales;
+    prm.y = y;
+    prm.M = M;
+    prm.N = N;
+    prm.K = K;
+    prm.bn = P.bn;
+    prm.xtiles = P.xtiles;
+    prm.idesc = prefill::make_idesc(prefill_ab::kRowsW, P.bn);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = P.grid;
+    cfg.blockDim = dim3(prefill_ab::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = prefill_ab::SmemLayout::total;
+    cfg.stream = stream;
+    return cudaLaunchKernelEx(&cfg, prefill_ab::prefill_ab_kernel, prm) == cudaSuccess ? W3_OK : W3_ERR_CUDA;
+}
+
 w3_status launch_decode(const uint16_t *x, const int32_t *packed, const uint16_t *scales, uint16_t *y, int M,
                         int N, int K, int num_sms, cudaStream_t stream) {
     const decode::LaunchPlan P = decode::plan(M, N, K, num_sms);
@@ -522,10 +585,14 @@ w3_status w3a16_gemm(const uint16_t *x, const int32_t *packed, const uint16_t *s
         if (partial && cudaFreeAsync(partial, st) != cudaSuccess && status == W3_OK) status = W3_ERR_CUDA;
         return status;
     }
-    // the prefill kernel's packed-word copies are 24 words wide: rows of at least 256 codes
-    if (M > 16 && W3_PREFILL_TCGEN05 && K >= 256)
+    // the prefill kernels' packed-word copies are 24 words wide: rows of at least 256 codes
+    if (M > 16 && W3_PREFILL_TCGEN05 && K >= 256) {
+        if (W3_PREFILL_SWAB && prefer_prefill_ab(static_cast<int>(M), static_cast<int>(N), sms))
+            return launch_prefill_ab(x, packed, scales, y, static_cast<int>(M), static_cast<int>(N),
+                                     static_cast<int>(K), st);
         return launch_prefill(x, packed, scales, y, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), sms,
                               st);
+    }
     // The tensor-core decode for N >= 256: one call per 16 batch rows, all sharing
     // one stream-ordered scratch buffer for the partial sums.
     const bool tc = N >= decode_tc::kRows && W3_DECODE_TC_MIN_M <= std::min<int64_t>(M, 16);

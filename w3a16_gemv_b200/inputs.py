@@ -146,4 +146,6 @@ def workloads() -> dict[str, Workload]:
     for name, n, k in LLAMA70B_LAYER:
         w[f"layer_{name}_m1"] = Workload(f"layer_{name}_m1", 1, n, k, "uniform8", "lognormal")
     w["prefill_2048x28672x8192"] = Workload("prefill_2048x28672x8192", 2048, 28672, 8192, "uniform8", "lognormal")
+    # a batch at which the tensor-memory prefill kernel is the one launched
+    w["prefill_1024x28672x8192"] = Workload("prefill_1024x28672x8192", 1024, 28672, 8192, "uniform8", "lognormal")
     return w
