@@ -12,7 +12,11 @@ bytes of one call are N*K*3/8 (packed) + N*K/128*2 (scales) + M*K*2 (x) +
 M*N*2 (y).  `roofline` is the dominant kernel's per-launch figure against the
 measured HBM copy bandwidth.  `e2e` is the same metric through the Python API
 with x copied from pinned host memory and y copied back every call.
-`cpu_baseline` times the CPU oracle on a bounded sample of the same step.
+`cpu_baseline` times the CPU oracle on a bounded sample of the same step, on
+every host core (OpenMP over rows) and on one.  `configs` adds, on one GPU,
+the other configurations: GEMV M=1 4096x4096, down_proj 8192x28672 at M=1 and
+8, the Llama-3.1-70B layer at M=1 (7 calls, and 4 row-concatenated calls in
+one CUDA graph) and the M=2048 prefill (tensor-core roofline).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 Under torchrun each rank runs an independent replica (the path does not shard);
@@ -41,28 +45,43 @@ BATCHES = (1, 4, 16)
 ROTATE = 5
 WORKLOAD = "Llama-3.1-70B gate_proj N=28672 K=8192, W3A16 g128 decode batch M=1,4,16"
 FALLBACK_HBM_GBS = 6650.0
-DECODE_SOURCES = ("w3a16_gemv_b200/csrc/decode_gemv.cuh", "w3a16_gemv_b200/csrc/decode_streamk.cuh",
-                  "w3a16_gemv_b200/csrc/decode_tcgen05.cuh", "w3a16_gemv_b200/csrc/prefill_gemm.cuh",
-                  "w3a16_gemv_b200/csrc/common.cuh")
+DECODE_SOURCES = ("w3a16_gemv_b200/csrc/api.cu", "w3a16_gemv_b200/csrc/decode_gemv.cuh",
+                  "w3a16_gemv_b200/csrc/decode_streamk.cuh", "w3a16_gemv_b200/csrc/decode_tcgen05.cuh",
+                  "w3a16_gemv_b200/csrc/prefill_gemm.cuh", "w3a16_gemv_b200/csrc/common.cuh")
 
 
 def algorithmic_bytes(M: int, N: int, K: int) -> int:
     return N * K * 3 // 8 + N * (K // 128) * 2 + M * K * 2 + M * N * 2
 
 
-def kernel_name(M: int) -> str:
-    """The kernel w3a16_gemm launches for a decode batch of M rows on the gate_proj shape."""
-    if M <= 4:
-        mt = 1 if M <= 1 else 2 if M <= 2 else 4
-        return f"w3::decode_sk::decode_sk_kernel<{mt}> (M={M})"
-    return f"w3::decode_tc::decode_tc_kernel (M={M})"
+# kernel symbol of each route of w3a16_gemm_route (the names in an ncu launch list)
+ROUTE_KERNELS = {
+    "decode_sk": "w3::decode_sk::decode_sk_kernel",
+    "decode": "w3::decode::decode_kernel",
+    "decode_tc": "w3::decode_tc::decode_tc_kernel",
+    "decode_tc32": "w3::decode_tc32::decode_tc_kernel",
+    "prefill": "w3::prefill::prefill_kernel",
+    "prefill_ab": "w3::prefill_ab::prefill_ab_kernel",
+    "passes": "16-row decode passes",
+}
 
 
-def kernels_per_call(M: int) -> int:
-    """Kernels w3a16_gemm launches for a decode batch of M rows on the gate_proj shape: the
-    tensor-core decode (M > 4) is followed by its partial-sum fix-up kernel (its work is split
-    over every SM, so some row tiles are shared)."""
-    return 1 if M <= 4 else 2
+def route(M: int, N: int, K: int, sms: int) -> str:
+    """The kernel route w3a16_gemm takes (asked from the library itself)."""
+    from w3a16_gemv_b200 import w3a16_gemm_route
+
+    return w3a16_gemm_route(M, N, K, num_sms=sms)
+
+
+def kernel_name(M: int, N: int, K: int, sms: int) -> str:
+    r = route(M, N, K, sms)
+    return f"{ROUTE_KERNELS.get(r, r)} (route {r}, M={M})"
+
+
+def kernels_per_call(M: int, N: int, K: int, sms: int) -> int:
+    """Kernels one w3a16_gemm call launches: the tensor-core decode routes are followed by their
+    partial-sum fix-up kernel when the work is split over more than one CTA (always, at these sizes)."""
+    return 2 if route(M, N, K, sms) in ("decode_tc", "decode_tc32") else 1
 
 
 def step_bytes() -> int:
@@ -193,31 +212,48 @@ def job_throughput(units_per_rank: float, world: int, max_ms: float) -> float:
 # CPU oracle (the reported baseline and the reference arm)
 # --------------------------------------------------------------------------------------
 
-def oracle_step_sample(budget_s: float):
-    """Time the oracle on the first rows of the step until `budget_s` of CPU work is spent.
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
 
-    Returns (GB/s in the metric's unit, seconds, rows, description)."""
+    return platform.processor() or "unknown"
+
+
+def oracle_step_sample(budget_s: float, threads: int | None = None):
+    """Time the oracle on slices of the step's weight rows until `budget_s` of wall time is spent.
+
+    threads: None = the plain single-threaded oracle; 0 = its OpenMP variant on every core (rows
+    spread over threads, each element the same k-ordered fp64 sum).
+    Returns (GB/s in the metric's unit, seconds, rows, threads used, description)."""
     import oracle
     from w3a16_gemv_b200.inputs import make_problem
 
     orc = oracle.get()
-    rows_per_chunk = 256
-    p = make_problem(max(BATCHES), rows_per_chunk, K_COLS, "uniform8", "lognormal", "normal", seed=0)
+    used = 1 if threads is None else (threads or orc.max_threads())
+    rows_per_chunk = 256 * used
+    p = make_problem(max(BATCHES), min(rows_per_chunk, N_ROWS), K_COLS, "uniform8", "lognormal", "normal", seed=0)
     packed = orc.pack(p.codes)
-    done_rows, spent, nbytes = 0, 0.0, 0
+    done_rows, spent = 0, 0.0
     while spent < budget_s and done_rows < N_ROWS:
         t0 = time.perf_counter()
         for m in BATCHES:
-            orc.gemm_f64(p.x_bf16[:m], packed, p.scales_bf16)
+            orc.gemm_f64(p.x_bf16[:m], packed, p.scales_bf16, threads=threads)
         spent += time.perf_counter() - t0
-        done_rows += rows_per_chunk
+        done_rows += p.N
     # bytes of the sampled rows in the metric's accounting (weights + the x/y share)
     frac = done_rows / N_ROWS
     nbytes = step_bytes() * frac
-    desc = (f"oracle_gemm_f64 (plain C, one thread) for M=1,4,16 over K=8192 on {done_rows} weight rows "
-            f"(a 256-row slice of the seeded workload, repeated; {frac:.2%} of one step's rows), "
-            f"GB/s = the step's algorithmic bytes scaled by rows / CPU seconds")
-    return nbytes / spent / 1e9, spent, done_rows, desc
+    how = "plain C, one thread" if threads is None else f"plain C with OpenMP over rows, {used} threads"
+    desc = (f"oracle_gemm_f64 ({how}) for M=1,4,16 over K=8192 on {done_rows} weight rows "
+            f"(a {p.N}-row slice of the seeded workload, repeated; {frac:.2%} of one step's rows), "
+            f"GB/s = the step's algorithmic bytes scaled by rows / wall seconds; CPU: {cpu_model()}")
+    return nbytes / spent / 1e9, spent, done_rows, used, desc
 
 
 def run_reference(args):
@@ -228,10 +264,10 @@ def run_reference(args):
     # keep the whole run within a few minutes whatever --steps/--warmup are
     budget = max(0.2, min(args.ref_budget, 150.0 / (args.steps + args.warmup)))
     for _ in range(args.warmup):
-        oracle_step_sample(min(0.5, budget))
-    desc = None
+        oracle_step_sample(min(0.5, budget), threads=0)
+    desc, used = None, 1
     for _ in range(args.steps):
-        gbs, spent, rows, desc = oracle_step_sample(budget)
+        gbs, spent, rows, used, desc = oracle_step_sample(budget, threads=0)
         per_step.append((gbs, spent))
     value = statistics.median(g for g, _ in per_step)
     line = {
@@ -240,7 +276,8 @@ def run_reference(args):
         "ms_per_step": statistics.median(1e3 * s for _, s in per_step), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": WORKLOAD, "sample": desc},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": used, "kind": "oracle", "sample": desc,
+                         "cpu_model": cpu_model()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -267,38 +304,11 @@ def measured_tensor_peak(sustained: bool = False):
         return 1590.0, "fallback (1.59 PFLOP/s earlier measurement on this pool)"
 
 
-def prefill_kernel_name(M: int, N: int, sms: int) -> str:
-    """The prefill kernel w3a16_gemm launches for M x N (M > 32): the same wave-cost rule as
-    api.cu (waves of 148 CTAs x per-wave time), used here only to label the roofline."""
-    import math
-
-    mt = (M + 255) // 256
-    best, best_eff = 256, -1.0
-    for bn in range(256, 127, -32):
-        tiles = mt * ((N + bn - 1) // bn)
-        waves = (tiles + sms - 1) // sms
-        eff = M * N / (waves * sms * 256 * bn)
-        if eff > best_eff + 1e-9:
-            best, best_eff = bn, eff
-    if N < 128:
-        best = (N + 31) // 32 * 32
-    cost_o = math.ceil(mt * ((N + best - 1) // best) / sms) * (43.0 + 0.27 * best)
-    bn_ab = 256 if M >= 256 else (M + 15) // 16 * 16
-    cost_a = math.ceil(((N + 127) // 128) * ((M + bn_ab - 1) // bn_ab) / sms) * 55.0
-    if M >= 256 and cost_a < 0.98 * cost_o:
-        return "w3::prefill_ab::prefill_ab_kernel"
-    return "w3::prefill::prefill_kernel"
-
-
-def run_prefill(args):
-    """Prefill workload: y = x W^T at M (default 2048), N=28672, K=8192 (one call per step)."""
+def _gpu_setup(world: int, local: int):
     import torch
 
     from w3a16_gemv_b200 import build as wbuild
-    from w3a16_gemv_b200 import w3_check_device_error, w3_pack, w3a16_gemm
-    from w3a16_gemv_b200.inputs import make_problem
 
-    world, rank, local = dist_setup()
     if world > 1:
         import torch.distributed as dist
 
@@ -308,63 +318,95 @@ def run_prefill(args):
     dev = torch.device("cuda", local)
     if not os.path.exists(wbuild.LIB):
         wbuild.build()
-    M, N, K = args.prefill_m, N_ROWS, K_COLS
+    return dev
+
+
+def measure_prefill(M: int, steps: int, warmup: int, dev, world: int = 1, sampler=None) -> dict:
+    """y = x W^T at M x 28672 x 8192 (one call per step), CUDA events around each call."""
+    import torch
+
+    from w3a16_gemv_b200 import w3_check_device_error, w3_pack, w3a16_gemm
+    from w3a16_gemv_b200.inputs import make_problem
+
+    N, K = N_ROWS, K_COLS
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
     p = make_problem(M, N, K, "uniform8", "lognormal", "normal", seed=0)
     packed = w3_pack(torch.from_numpy(p.codes).to(dev))
     scales = torch.from_numpy(p.scales_bf16.view(np.int16)).view(torch.bfloat16).to(dev)
     x = torch.from_numpy(p.x_bf16.view(np.int16)).view(torch.bfloat16).to(dev)
     y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream()
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         w3a16_gemm(x, packed, scales, out=y)
     torch.cuda.synchronize()
     w3_check_device_error()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    sampler = ClockSampler(local)
-    sampler.start()
-    time.sleep(0.02)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
     w0 = time.perf_counter()
-    for i in range(args.steps):
+    for i in range(steps):
         ev[i][0].record(stream)
         w3a16_gemm(x, packed, scales, out=y)
         ev[i][1].record(stream)
     torch.cuda.synchronize()
     w1 = time.perf_counter()
-    sampler.stop()
     w3_check_device_error()
     per_ms = [a.elapsed_time(b) for a, b in ev]
-    total_ms = ev[0][0].elapsed_time(ev[-1][1])
-    total_ms = max_over_ranks(total_ms, world, dev)
+    total_ms = max_over_ranks(ev[0][0].elapsed_time(ev[-1][1]), world, dev)
     flop = 2.0 * M * N * K
-    value = job_throughput(flop * args.steps, world, total_ms) / 1e12
     # a timed region of half a second or more runs the tensor cores under the power cap: compare with
     # the sustained figure; a short one with the burst figure
     peak, src = measured_tensor_peak(sustained=total_ms >= 500.0)
     achieved = flop / (statistics.mean(per_ms) * 1e-3) / 1e12
-    sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    line = {
-        "metric": f"W3A16 g128 prefill GEMM TFLOP/s (M={M}, Llama-70B gate_proj)", "value": value,
-        "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": f"prefill M={M} N={N} K={K} (Llama-3.1-70B gate_proj)", "M": M, "N": N, "K": K,
-                   "l2": f"inputs larger than L2 (x {M * K * 2 / 1e6:.1f} MB + weights {N * K * 3 / 8e6:.1f} MB"
-                         f" + y {M * N * 2 / 1e6:.1f} MB)"},
-        "us_per_call": 1e3 * statistics.median(per_ms),
+    rec = {
+        "workload": f"prefill M={M} N={N} K={K} (Llama-3.1-70B gate_proj), codes uniform 0..7, "
+                    "scales bf16 lognormal(-4, 0.5), x bf16 N(0,1)",
+        "M": M, "N": N, "K": K, "steps": steps, "total_ms": total_ms,
+        "us_per_call": 1e3 * statistics.median(per_ms), "us_mean": 1e3 * statistics.mean(per_ms),
+        "TFLOP/s": job_throughput(flop * steps, world, total_ms) / 1e12,
+        "GB/s": algorithmic_bytes(M, N, K) / (statistics.mean(per_ms) * 1e-3) / 1e9,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": None, "kernel": prefill_kernel_name(M, N, sms),
+                     "frac": achieved / peak, "traffic": None, "kernel": kernel_name(M, N, K, sms),
                      "peak_source": src, "frac_of_nominal_2250": achieved / 2250.0},
-        "gpu_launches": args.steps,
-        "clocks": sampler.summary(w0, w1),
+        "l2": f"inputs larger than L2 (x {M * K * 2 / 1e6:.1f} MB + weights {N * K * 3 / 8e6:.1f} MB"
+              f" + y {M * N * 2 / 1e6:.1f} MB)",
+    }
+    if sampler is not None:
+        rec["clocks"] = sampler.summary(w0, w1)
+    return rec
+
+
+def run_prefill(args):
+    """Prefill workload: y = x W^T at M (default 2048), N=28672, K=8192 (one call per step)."""
+    world, rank, local = dist_setup()
+    dev = _gpu_setup(world, local)
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.02)
+    rec = measure_prefill(args.prefill_m, args.steps, args.warmup, dev, world, sampler)
+    sampler.stop()
+    M = args.prefill_m
+    line = {
+        "metric": f"W3A16 g128 prefill GEMM TFLOP/s (M={M}, Llama-70B gate_proj)", "value": rec["TFLOP/s"],
+        "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": rec["total_ms"] / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": rec["workload"], "M": M, "N": N_ROWS, "K": K_COLS, "l2": rec["l2"]},
+        "us_per_call": rec["us_per_call"], "roofline": rec["roofline"], "gpu_launches": args.steps,
+        "clocks": rec.get("clocks"),
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
-        torch.distributed.destroy_process_group()
+        torch_dist_done()
     return 0
+
+
+def torch_dist_done():
+    import torch
+
+    torch.distributed.destroy_process_group()
 
 
 SWEEPS = {
@@ -379,24 +421,39 @@ SWEEPS = {
 }
 
 
-def run_sweep(args):
-    """Per-call timing of the other decode configurations (one GPU): each call's weights rotate
-    among enough copies that every call streams them from HBM; for the layer sweep, also one CUDA
-    graph of the seven calls replayed `steps` times."""
+def _graph_us(calls_of_copy, copies: int, reps: int, stream) -> float:
+    """Device time per call: one CUDA graph holding the call on every weight copy, replayed."""
     import torch
 
-    from w3a16_gemv_b200 import build as wbuild
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for r in range(copies):
+            calls_of_copy(r)
+    g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(reps):
+        g.replay()
+    b.record(stream)
+    torch.cuda.synchronize()
+    us = a.elapsed_time(b) * 1e3 / (reps * copies)
+    del g
+    return us
+
+
+def measure_sweep(name: str, steps: int, warmup: int, dev, sampler=None) -> dict:
+    """Per-call timing of one of the other decode configurations (one GPU): each call's weights
+    rotate among enough copies that every call streams them from HBM; device time per call from a
+    replayed CUDA graph of the call over its copies; for the layer sweep, also one CUDA graph of the
+    seven calls and the 4-call fused layer."""
+    import torch
+
     from w3a16_gemv_b200 import w3_check_device_error, w3_pack, w3a16_gemm
     from w3a16_gemv_b200.inputs import workloads
 
-    world, rank, local = dist_setup()
-    if rank != 0:
-        return 0
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if not os.path.exists(wbuild.LIB):
-        wbuild.build()
-    desc, names = SWEEPS[args.workload]
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    desc, names = SWEEPS[name]
     wls = [workloads()[n] for n in names]
     pass_bytes = sum(algorithmic_bytes(0, w.N, w.K) for w in wls)
     copies = max(2, -(-3 * 126_000_000 // pass_bytes))  # more than three L2 sizes in rotation
@@ -420,72 +477,52 @@ def run_sweep(args):
             if ev is not None:
                 ev[j][1].record(stream)
 
-    for i in range(args.warmup):
+    for i in range(warmup):
         one_pass(i)
     torch.cuda.synchronize()
     w3_check_device_error()
     events = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)] for _ in calls]
-              for _ in range(args.steps)]
-    sampler = ClockSampler(local)
-    sampler.start()
-    time.sleep(0.02)
+              for _ in range(steps)]
     torch.cuda.synchronize()
     w0 = time.perf_counter()
-    for i in range(args.steps):
-        one_pass(args.warmup + i, events[i])
+    for i in range(steps):
+        one_pass(warmup + i, events[i])
     torch.cuda.synchronize()
     w1 = time.perf_counter()
-    sampler.stop()
     w3_check_device_error()
-    # device time per call without host overhead: a CUDA graph of the call on every weight copy, replayed
-    graph_us = []
-    reps = max(3, args.steps // copies)
-    for c in calls:
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            for r in range(copies):
-                w3a16_gemm(c["x"], c["packs"][r], c["scales"][r], out=c["y"])
-        g.replay()
-        torch.cuda.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(reps):
-            g.replay()
-        b.record(stream)
-        torch.cuda.synchronize()
-        graph_us.append(a.elapsed_time(b) * 1e3 / (reps * copies))
-        del g
+    reps = max(3, steps // copies)
+    graph_us = [_graph_us(lambda r, c=c: w3a16_gemm(c["x"], c["packs"][r], c["scales"][r], out=c["y"]),
+                          copies, reps, stream) for c in calls]
     w3_check_device_error()
     peak, peak_src = measured_peak()
     out_calls, total_us, total_bytes = [], 0.0, 0
     for j, c in enumerate(calls):
         w = c["w"]
-        ts = np.array([events[i][j][0].elapsed_time(events[i][j][1]) for i in range(args.steps)]) * 1e3
+        ts = np.array([events[i][j][0].elapsed_time(events[i][j][1]) for i in range(steps)]) * 1e3
         med = float(np.median(ts))
         b = algorithmic_bytes(w.M, w.N, w.K)
         total_us += med
         total_bytes += b
         gu = graph_us[j]
-        out_calls.append({"name": w.name, "M": w.M, "N": w.N, "K": w.K,
+        out_calls.append({"name": w.name, "M": w.M, "N": w.N, "K": w.K, "kernel": kernel_name(w.M, w.N, w.K, sms),
                           "us_median": med, "us_p10": float(np.percentile(ts, 10)),
                           "us_p90": float(np.percentile(ts, 90)), "us_device_graph": gu,
                           "GB/s": b / (gu * 1e-6) / 1e9, "frac_of_peak": b / (gu * 1e-6) / 1e9 / peak,
                           "TFLOP/s": 2.0 * w.M * w.N * w.K / (gu * 1e-6) / 1e12})
-    line = {
-        "metric": METRIC, "value": total_bytes / (sum(graph_us) * 1e-6) / 1e9, "unit": UNIT, "n_gpus": 1,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sum(graph_us) / 1e3, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": desc, "calls": list(names),
-                   "l2": f"inputs larger than L2: {copies} rotating copies of every call's weights "
-                         f"({copies * pass_bytes / 1e6:.0f} MB)"},
-        "sum_of_median_us": total_us, "sum_of_device_us": sum(graph_us),
+    rec = {
+        "workload": desc, "calls_list": list(names), "GB/s": total_bytes / (sum(graph_us) * 1e-6) / 1e9,
+        "frac_of_peak": total_bytes / (sum(graph_us) * 1e-6) / 1e9 / peak,
+        "sum_of_median_us": total_us, "sum_of_device_us": sum(graph_us), "steps": steps,
+        "l2": f"inputs larger than L2: {copies} rotating copies of every call's weights "
+              f"({copies * pass_bytes / 1e6:.0f} MB)",
         "timing": "us_median/p10/p90: CUDA events around each call (include host launch overhead when the "
                   "kernel is shorter than it); us_device_graph and GB/s: one CUDA graph of the call on every "
                   "weight copy, replayed, time per call",
         "calls": out_calls, "peak": peak, "peak_source": peak_src,
-        "clocks": sampler.summary(w0, w1),
     }
-    if args.workload == "layer":
+    if sampler is not None:
+        rec["clocks"] = sampler.summary(w0, w1)
+    if name == "layer":
         # one CUDA graph of the seven calls on fixed copies, replayed
         g = torch.cuda.CUDAGraph()
         side = torch.cuda.Stream()
@@ -501,21 +538,44 @@ def run_sweep(args):
         torch.cuda.synchronize()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        for _ in range(args.steps):
+        for _ in range(steps):
             g.replay()
         b.record(stream)
         torch.cuda.synchronize()
         w3_check_device_error()
-        g_us = a.elapsed_time(b) * 1e3 / args.steps
-        line["cuda_graph"] = {"us_per_replay": g_us, "GB/s": total_bytes / (g_us * 1e-6) / 1e9,
-                              "note": "weights of one copy, 7 calls per replay (L2 holds part of them)"}
+        g_us = a.elapsed_time(b) * 1e3 / steps
+        rec["cuda_graph"] = {"us_per_replay": g_us, "GB/s": total_bytes / (g_us * 1e-6) / 1e9,
+                             "note": "weights of one copy, 7 calls per replay (L2 holds part of them)"}
         del g
-        line["fused"] = fused_layer(calls, copies, args, stream, total_bytes)
+        rec["fused"] = fused_layer(calls, copies, steps, stream, total_bytes)
+    return rec
+
+
+def run_sweep(args):
+    import torch
+
+    world, rank, local = dist_setup()
+    if rank != 0:
+        return 0
+    torch.cuda.set_device(local)
+    dev = _gpu_setup(1, local)
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.02)
+    rec = measure_sweep(args.workload, args.steps, args.warmup, dev, sampler)
+    sampler.stop()
+    line = {
+        "metric": METRIC, "value": rec["GB/s"], "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": rec["sum_of_device_us"] / 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": rec["workload"], "calls": rec["calls_list"], "l2": rec["l2"]},
+    }
+    line.update({k: v for k, v in rec.items() if k not in ("workload", "calls_list", "l2", "GB/s")})
     print(json.dumps(line), flush=True)
     return 0
 
 
-def fused_layer(calls, copies, args, stream, total_bytes):
+def fused_layer(calls, copies, steps, stream, total_bytes):
     """The same layer as 4 calls: q, k, v and gate, up concatenated along N (rows of the format
     are independent, so a row-concatenated packed/scales pair is one weight), o and down alone.
     Device time of each call from graph replays over its copies, and one graph of the 4 calls."""
@@ -536,26 +596,14 @@ def fused_layer(calls, copies, args, stream, total_bytes):
               cat(["layer_gate_proj_m1", "layer_up_proj_m1"]), cat(["layer_down_proj_m1"])]
     for c in fcalls:
         c["y"] = torch.empty((1, c["N"]), dtype=torch.bfloat16, device=c["x"].device)
-    reps = max(3, args.steps // copies)
+    reps = max(3, steps // copies)
     out = []
     for c in fcalls:
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            for r in range(copies):
-                w3a16_gemm(c["x"], c["packs"][r], c["scales"][r], out=c["y"])
-        g.replay()
-        torch.cuda.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(reps):
-            g.replay()
-        b.record(stream)
-        torch.cuda.synchronize()
-        us = a.elapsed_time(b) * 1e3 / (reps * copies)
+        us = _graph_us(lambda r, c=c: w3a16_gemm(c["x"], c["packs"][r], c["scales"][r], out=c["y"]), copies, reps,
+                       stream)
         byt = algorithmic_bytes(1, c["N"], c["K"])
         out.append({"name": c["name"], "N": c["N"], "K": c["K"], "us_device_graph": us,
                     "GB/s": byt / (us * 1e-6) / 1e9})
-        del g
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
         for c in fcalls:
@@ -565,12 +613,12 @@ def fused_layer(calls, copies, args, stream, total_bytes):
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
-    for _ in range(args.steps):
+    for _ in range(steps):
         g.replay()
     b.record(stream)
     torch.cuda.synchronize()
     w3_check_device_error()
-    g_us = a.elapsed_time(b) * 1e3 / args.steps
+    g_us = a.elapsed_time(b) * 1e3 / steps
     del g
     return {"calls": out, "sum_of_device_us": sum(c["us_device_graph"] for c in out),
             "cuda_graph_us_per_replay": g_us, "GB/s": total_bytes / (g_us * 1e-6) / 1e9}
@@ -579,20 +627,12 @@ def fused_layer(calls, copies, args, stream, total_bytes):
 def run_gpu(args):
     import torch
 
-    from w3a16_gemv_b200 import build as wbuild
     from w3a16_gemv_b200 import w3_check_device_error, w3_pack, w3a16_gemm
     from w3a16_gemv_b200.inputs import make_problem
 
     world, rank, local = dist_setup()
-    if world > 1:
-        import torch.distributed as dist
-
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if not os.path.exists(wbuild.LIB):
-        wbuild.build()
+    dev = _gpu_setup(world, local)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
 
     # ---- inputs: seeded, drawn on the host, packed on the device by w3_pack ----
     p = make_problem(max(BATCHES), N_ROWS, K_COLS, "uniform8", "lognormal", "normal", seed=0)
@@ -643,18 +683,19 @@ def run_gpu(args):
     w1 = time.perf_counter()
     if world > 1:
         torch.distributed.barrier()
-    sampler.stop()
     w3_check_device_error()
     elapsed_ms = t_start.elapsed_time(t_end)
 
-    # ---- per-call breakdown (second timed pass): an event pair around every call, which also
-    #      keeps consecutive calls from overlapping; the roofline's per-launch time comes from here ----
-    brk_steps = min(args.steps, 500)
+    # ---- per-call breakdown (second timed pass, at least 200 steps): an event pair around every
+    #      call, which also keeps consecutive calls from overlapping; the roofline's per-launch time
+    #      comes from here ----
+    brk_steps = max(200, min(args.steps, 500))
     events = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
                for _ in BATCHES] for _ in range(brk_steps)]
     for i in range(brk_steps):
         one_step(args.warmup + args.steps + i, events[i])
     torch.cuda.synchronize()
+    sampler.stop()
     w3_check_device_error()
     per_call_ms = {m: [events[i][j][0].elapsed_time(events[i][j][1]) for i in range(brk_steps)]
                    for j, m in enumerate(BATCHES)}
@@ -670,7 +711,8 @@ def run_gpu(args):
         us = 1e3 * statistics.mean(per_call_ms[m])
         b = algorithmic_bytes(m, N_ROWS, K_COLS)
         q = np.percentile(np.array(per_call_ms[m]) * 1e3, [10, 90])
-        calls.append({"M": m, "us_mean": us, "us_median": 1e3 * statistics.median(per_call_ms[m]),
+        calls.append({"M": m, "kernel": kernel_name(m, N_ROWS, K_COLS, sms), "us_mean": us,
+                      "us_median": 1e3 * statistics.median(per_call_ms[m]),
                       "us_p10": float(q[0]), "us_p90": float(q[1]),
                       "GB/s": b / (us * 1e-6) / 1e9, "TFLOP/s": 2.0 * m * N_ROWS * K_COLS / (us * 1e-6) / 1e12,
                       "frac_of_peak": b / (us * 1e-6) / 1e9 / peak, "share": 0.0})
@@ -678,11 +720,11 @@ def run_gpu(args):
     for c in calls:
         c["share"] = c["us_mean"] / tot
     dom = max(calls, key=lambda c: c["us_mean"])
-    traffic = recorded_traffic(dom["M"])
     roofline = {"bound": "hbm", "achieved": dom["GB/s"], "peak": peak, "unit": "GB/s",
-                "frac": dom["GB/s"] / peak, "traffic": traffic,
-                "kernel": kernel_name(dom["M"]),
+                "frac": dom["GB/s"] / peak, "traffic": recorded_traffic(dom["M"]),
+                "kernel": dom["kernel"],
                 "algorithmic_bytes_per_launch": algorithmic_bytes(dom["M"], N_ROWS, K_COLS),
+                "launch_time": f"mean of {brk_steps} CUDA-event pairs around the call, on the launch stream",
                 "peak_source": peak_src}
 
     # ---- end to end through the public API with host buffers ----
@@ -738,19 +780,36 @@ def run_gpu(args):
         "calls": calls,
         "roofline": roofline,
         "e2e": e2e,
-        "gpu_launches": args.steps * sum(kernels_per_call(m) for m in BATCHES),
+        "gpu_launches": args.steps * sum(kernels_per_call(m, N_ROWS, K_COLS, sms) for m in BATCHES),
         "per_call_timing": f"calls[]: CUDA events around each call over {brk_steps} further steps (no overlap "
                            "between calls); value: the K steps back to back",
         "clocks": clocks,
     }
+    del packs, scales, x_all, xs, ys, x_dev, y_dev
+    torch.cuda.empty_cache()
+    if rank == 0 and world == 1 and not args.no_configs:
+        # the other configurations, each on its own inputs (one GPU; device time per call)
+        cs = ClockSampler(local)
+        cs.start()
+        time.sleep(0.02)
+        configs = {"1_gemv_4096": measure_sweep("gemv4096", 50, 5, dev, cs),
+                   "2_gate_decode": {"workload": WORKLOAD, "see": "value, calls, roofline of this line"},
+                   "3_down_proj": measure_sweep("down", 50, 5, dev, cs),
+                   "4_layer": measure_sweep("layer", 50, 5, dev, cs),
+                   "5_prefill_2048": measure_prefill(2048, 20, 3, dev, 1, cs)}
+        cs.stop()
+        line["configs"] = configs
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        gbs, spent, rows, desc = oracle_step_sample(args.cpu_budget)
-        line["cpu_baseline"] = {"value": gbs, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc,
-                                "seconds": spent}
+        gbs1, spent1, rows1, _, desc1 = oracle_step_sample(args.cpu_budget / 2)
+        gbsn, spentn, rowsn, used, descn = oracle_step_sample(args.cpu_budget / 2, threads=0)
+        line["cpu_baseline"] = {"value": gbsn, "unit": UNIT, "cores": used, "kind": "oracle", "sample": descn,
+                                "seconds": spentn, "cpu_model": cpu_model(), "os_cpu_count": os.cpu_count(),
+                                "single_core": {"value": gbs1, "unit": UNIT, "cores": 1, "sample": desc1,
+                                                "seconds": spent1}}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
-        torch.distributed.destroy_process_group()
+        torch_dist_done()
     return 0
 
 
@@ -763,6 +822,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of CPU oracle work for cpu_baseline")
     ap.add_argument("--ref-budget", type=float, default=3.0, help="seconds of oracle work per reference step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the other configurations (GEMV 4096, down_proj, 70B layer, M=2048 prefill)")
     ap.add_argument("--prefill-m", type=int, default=2048, help="batch rows of the prefill workload (M > 32)")
     ap.add_argument("--workload", choices=("gate_decode", "prefill") + tuple(SWEEPS), default="gate_decode",
                     help="gate_decode: the headline decode step (default); prefill: M=2048 tensor-core GEMM; "

@@ -157,6 +157,24 @@ w3_status w3a16_gemm_noalloc(const uint16_t *x, const int32_t *packed, const uin
                              int64_t M, int64_t N, int64_t K, w3_stream_t stream);
 
 /*
+ * w3a16_gemm_route -- which kernels w3a16_gemm (and w3a16_gemm_noalloc) run for
+ * an M x N x K product on a GPU with `num_sms` SMs, as a short name:
+ *   "decode_sk"   persistent stream-K mma.sync decode (M <= 4, many rows);
+ *   "decode"      mma.sync decode with cluster split-K (the other M <= 16 shapes);
+ *   "decode_tc"   tensor-core (tcgen05) decode, 16 columns (5 <= M <= 16, N >= 256);
+ *   "decode_tc32" the same, 32 columns (17 <= M <= 32, N >= 256);
+ *   "prefill"     tcgen05 GEMM, weights dequantized into shared memory;
+ *   "prefill_ab"  tcgen05 GEMM, weights dequantized into tensor memory;
+ *   "passes"      M > 16 with K < 256: the decode routes on 16-row slices of x.
+ * The choice depends only on the shape and the SM count (no device is touched,
+ * so it can be asked on a machine without a GPU).  Returns NULL for a shape
+ * that w3a16_gemm rejects with W3_ERR_SHAPE, or num_sms < 1.  The string is
+ * static; do not free it.  No counterpart in the format's pages: it names this
+ * library's kernels.
+ */
+const char *w3a16_gemm_route(int64_t M, int64_t N, int64_t K, int32_t num_sms);
+
+/*
  * w3_check_device_error -- synchronise `stream`, then report and clear the
  * current device's error flag: W3_OK, or W3_ERR_TIMEOUT if a kernel of this
  * library gave up a bounded wait since the last check.  W3_ERR_CUDA if the

@@ -41,7 +41,7 @@ def build(force: bool = False) -> str:
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
         tmp = _LIB + f".tmp{os.getpid()}"
         subprocess.check_call(
-            ["gcc", "-O2", "-std=c11", "-Wall", "-Wextra", "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"]
+            ["gcc", "-O2", "-std=c11", "-Wall", "-Wextra", "-fPIC", "-fopenmp", "-shared", "-o", tmp, _SRC, "-lm"]
         )
         os.replace(tmp, _LIB)
     return _LIB
@@ -67,6 +67,10 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         lib.oracle_dequant_f32.restype = ctypes.c_int
         lib.oracle_gemm_f64.argtypes = [p, p, p, p, i64, i64, i64]
         lib.oracle_gemm_f64.restype = ctypes.c_int
+        lib.oracle_gemm_f64_threads.argtypes = [p, p, p, p, i64, i64, i64, ctypes.c_int]
+        lib.oracle_gemm_f64_threads.restype = ctypes.c_int
+        lib.oracle_max_threads.argtypes = []
+        lib.oracle_max_threads.restype = ctypes.c_int
         lib.oracle_gemm_f64_entries.argtypes = [p, p, p, i64, i64, i64, p, p, i64, p]
         lib.oracle_gemm_f64_entries.restype = ctypes.c_int
         lib.oracle_weight_row_norms.argtypes = [p, p, i64, i64, p]
@@ -161,8 +165,14 @@ class Oracle:
                "oracle_dequant_f32")
         return out
 
-    def gemm_f64(self, x_bf16: np.ndarray, packed: np.ndarray, scales_bf16: np.ndarray) -> np.ndarray:
-        """y = x W^T in fp64, [M,N]."""
+    def max_threads(self) -> int:
+        """Threads a multi-threaded call uses by default (all cores)."""
+        return int(self.lib.oracle_max_threads())
+
+    def gemm_f64(self, x_bf16: np.ndarray, packed: np.ndarray, scales_bf16: np.ndarray,
+                 threads: int | None = None) -> np.ndarray:
+        """y = x W^T in fp64, [M,N].  threads: None = one thread; 0 = all cores; n = n threads
+        (rows n spread over threads; every element is the same k-ordered fp64 sum)."""
         x_bf16 = _c(x_bf16.view(np.uint16), np.uint16)
         packed = _c(packed.view(np.uint32), np.uint32)
         scales_bf16 = _c(scales_bf16.view(np.uint16), np.uint16)
@@ -170,8 +180,12 @@ class Oracle:
         N = packed.shape[0]
         self._shapes(packed, scales_bf16, N, K)
         out = np.empty((M, N), dtype=np.float64)
-        _check(self.lib.oracle_gemm_f64(_ptr(x_bf16), _ptr(packed), _ptr(scales_bf16), _ptr(out), M, N, K),
-               "oracle_gemm_f64")
+        if threads is None:
+            _check(self.lib.oracle_gemm_f64(_ptr(x_bf16), _ptr(packed), _ptr(scales_bf16), _ptr(out), M, N, K),
+                   "oracle_gemm_f64")
+        else:
+            _check(self.lib.oracle_gemm_f64_threads(_ptr(x_bf16), _ptr(packed), _ptr(scales_bf16), _ptr(out),
+                                                    M, N, K, int(threads)), "oracle_gemm_f64_threads")
         return out
 
     def gemm_f64_entries(self, x_bf16, packed, scales_bf16, ms, ns) -> np.ndarray:

@@ -42,6 +42,9 @@
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 
 #define ORACLE_GROUP 128
 
@@ -160,6 +163,52 @@ int oracle_gemm_f64(const uint16_t *x, const uint32_t *packed, const uint16_t *s
     }
     free(wrow);
     return 0;
+}
+
+/*
+ * The same y as oracle_gemm_f64, with the output rows n spread over `threads`
+ * OpenMP threads (0: the OpenMP default, all cores).  Every element is still
+ * one fp64 dot product in ascending k computed by one thread, so the result is
+ * bit-identical to oracle_gemm_f64; only the wall time changes.
+ */
+int oracle_gemm_f64_threads(const uint16_t *x, const uint32_t *packed, const uint16_t *scales,
+                            double *y, int64_t M, int64_t N, int64_t K, int threads) {
+    if (!x || !packed || !scales || !y || M < 0 || N < 0 || threads < 0) return -1;
+    if (oracle_words_per_row(K) < 0 || oracle_groups_per_row(K) < 0) return -1;
+    int failed = 0;
+#ifdef _OPENMP
+    const int nt = threads > 0 ? threads : omp_get_max_threads();
+#pragma omp parallel num_threads(nt)
+#endif
+    {
+        float *wrow = (float *)malloc((size_t)K * sizeof(float));
+        if (!wrow) {
+#ifdef _OPENMP
+#pragma omp atomic write
+#endif
+            failed = 1;
+        }
+#ifdef _OPENMP
+#pragma omp for schedule(dynamic, 16)
+#endif
+        for (int64_t n = 0; n < N; ++n) {
+            if (!wrow) continue;
+            dequant_row(packed, scales, n, K, wrow);
+            for (int64_t m = 0; m < M; ++m)
+                y[m * N + n] = dot_row(x, wrow, m, K);
+        }
+        free(wrow);
+    }
+    return failed ? -1 : 0;
+}
+
+/* Threads oracle_gemm_f64_threads(..., 0) uses: the OpenMP default (1 without OpenMP). */
+int oracle_max_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
 }
 
 /*

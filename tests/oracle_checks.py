@@ -147,6 +147,10 @@ def check_group_scales_exact(orc):
 
 # --- the product ----------------------------------------------------------------------
 
+# The single-threaded product and its multi-threaded variant (rows spread over threads) are
+# both held to every pin of the product.
+PRODUCT_THREADS = (None, 2)
+
 def check_brute_force_tiny(orc):
     rng = np.random.Generator(np.random.PCG64(5))
     for M, N, K in [(1, 1, 128), (2, 3, 128), (2, 3, 256), (3, 2, 384)]:
@@ -154,13 +158,14 @@ def check_brute_force_tiny(orc):
         codes = rng.integers(0, 8, size=(N, K), dtype=np.uint8)
         xi = rng.integers(-8, 9, size=(M, K))
         se = rng.integers(-4, 3, size=(N, G))
-        y = orc.gemm_f64(_bf16(xi), orc.pack(codes), _bf16(np.ldexp(1.0, se)))
-        assert y.shape == (M, N)
-        for m in range(M):
-            for n in range(N):
-                exact = sum(Fraction(int(xi[m, k])) * (int(codes[n, k]) - 4) * Fraction(2) ** int(se[n, k // 128])
-                            for k in range(K))
-                assert Fraction(y[m, n]) == exact, (M, N, K, m, n)
+        for threads in PRODUCT_THREADS:
+            y = orc.gemm_f64(_bf16(xi), orc.pack(codes), _bf16(np.ldexp(1.0, se)), threads=threads)
+            assert y.shape == (M, N)
+            for m in range(M):
+                for n in range(N):
+                    exact = sum(Fraction(int(xi[m, k])) * (int(codes[n, k]) - 4) *
+                                Fraction(2) ** int(se[n, k // 128]) for k in range(K))
+                    assert Fraction(y[m, n]) == exact, (M, N, K, m, n, threads)
 
 
 def check_position_probe(orc):
@@ -171,10 +176,11 @@ def check_position_probe(orc):
     s = bf16_bits_to_f32(scales).astype(np.float64)
     packed = orc.pack(codes)
     eye = np.eye(K, dtype=np.float32)
-    y = orc.gemm_f64(_bf16(eye), packed, scales)  # row k of x is e_k
-    for k in range(K):
-        for n in range(N):
-            assert y[k, n] == (int(codes[n, k]) - 4) * s[n, k // 128], (k, n)
+    for threads in PRODUCT_THREADS:
+        y = orc.gemm_f64(_bf16(eye), packed, scales, threads=threads)  # row k of x is e_k
+        for k in range(K):
+            for n in range(N):
+                assert y[k, n] == (int(codes[n, k]) - 4) * s[n, k // 128], (k, n, threads)
 
 
 def check_closed_forms(orc):
@@ -192,8 +198,14 @@ def check_closed_forms(orc):
             assert np.all(y[m] == (c - 4) * s * int(xi[m].sum()))
     # x = 1, s = 1 -> y[0,n] = sum_k q[n,k]
     codes = rng.integers(0, 8, size=(N, K), dtype=np.uint8)
-    y = orc.gemm_f64(_bf16(np.ones((1, K))), orc.pack(codes), _bf16(np.ones((N, K // 128))))
-    assert np.array_equal(y[0], np.array([int(codes[n].astype(np.int64).sum()) - 4 * K for n in range(N)], float))
+    for threads in PRODUCT_THREADS:
+        y = orc.gemm_f64(_bf16(np.ones((1, K))), orc.pack(codes), _bf16(np.ones((N, K // 128))), threads=threads)
+        assert np.array_equal(y[0], np.array([int(codes[n].astype(np.int64).sum()) - 4 * K for n in range(N)],
+                                             float))
+    # the multi-threaded product on a constant code
+    y = orc.gemm_f64(x, orc.pack(np.full((N, K), 7, np.uint8)), _bf16(np.full((N, K // 128), 0.25)), threads=3)
+    for m in range(M):
+        assert np.all(y[m] == 3 * 0.25 * int(xi[m].sum()))
 
 
 def check_numpy_cross_check(orc):
@@ -207,6 +219,8 @@ def check_numpy_cross_check(orc):
     ref = X @ W.T
     y = orc.gemm_f64(x, orc.pack(codes), scales)
     assert np.all(np.abs(y - ref) <= 1e-12 * (np.abs(X) @ np.abs(W).T) + 1e-300)
+    yt = orc.gemm_f64(x, orc.pack(codes), scales, threads=3)
+    assert np.all(np.abs(yt - ref) <= 1e-12 * (np.abs(X) @ np.abs(W).T) + 1e-300)
     # sampled entries agree with the full product bit for bit
     ms, ns = rng.integers(0, M, 50), rng.integers(0, N, 50)
     assert np.array_equal(orc.gemm_f64_entries(x, orc.pack(codes), scales, ms, ns), y[ms, ns])

@@ -4,8 +4,12 @@
 * y = x W^T: every checked element within |y - y_ref| <= 1e-2*||x_m||*||w_n||/sqrt(K) + 1e-3
   of the fp64 oracle.
 Small shapes are checked in full (several tiles, ragged edges, every decode
-batch size); the full-size workloads are checked on sampled outputs computed
-one by one by the oracle, in the same launch configuration the benchmark times.
+batch size).  The full-size decode workloads (every M <= 16 configuration the
+benchmark times) are checked in full against the oracle; the M = 2048 and
+M = 1024 prefill workloads on 64 whole rows of y plus 4096 sampled entries.
+Position probes (x = e_k) go through every kernel route, each asserted with
+w3a16_gemm_route, so that a bit-order or placement mistake in any one kernel
+shows up as a wrong weight in a known place.
 """
 import numpy as np
 import pytest
@@ -13,7 +17,8 @@ import torch
 
 import oracle
 from gpu_helpers import assert_within_bound, bound, device_problem, from_dev_bf16
-from w3a16_gemv_b200 import build, w3_check_device_error, w3_dequant_f32, w3_pack, w3_unpack, w3a16_gemm
+from w3a16_gemv_b200 import (build, w3_check_device_error, w3_dequant_f32, w3_pack, w3_unpack, w3a16_gemm,
+                             w3a16_gemm_route)
 from w3a16_gemv_b200.inputs import make_problem, workloads
 
 pytestmark = pytest.mark.gpu
@@ -67,6 +72,9 @@ SMALL = [
     (20, 1000, 4224, "gsq_5level", "absnormal", "normal_outliers"),
     (24, 28672, 256, "uniform8", "lognormal", "normal"),          # many row tiles, two groups
     (31, 300, 8192, "uniform8", "lognormal", "normal"),
+    # the shared-memory prefill with a ragged second 128-row batch tile and a ragged last W tile
+    (200, 1000, 1024, "gsq_5level", "absnormal", "normal_outliers"),
+    (129, 600, 512, "uniform8", "lognormal", "normal"),
 ]
 
 
@@ -132,36 +140,45 @@ def test_batch_rows_match_single_row_calls(orc):
     print(f"batch-invariance: {same}/16 rows bit-identical between M=1 and M=16")
 
 
-def test_position_probe_32_wide(orc):
-    # 32 batch rows, each a unit vector: every column of the 32-wide decode picks one weight
-    N, K = 300, 512
-    p = make_problem(32, N, K, seed=16)
+def _probe(orc, M, N, K, seed):
+    """x = e_k in every batch row (row i picks column k0 + i): y[i, n] must be the dequantized
+    weight W[n, k0 + i] rounded once to bf16, for every n and every k."""
+    p = make_problem(M, N, K, seed=seed)
     _, codes, scales = device_problem(p)
     packed = w3_pack(codes)
     w = orc.dequant_f32(orc.pack(p.codes), p.scales_bf16, K)
-    for k0 in range(0, K, 32):
-        eye = np.zeros((32, K), dtype=np.float32)
-        eye[np.arange(32), k0 + np.arange(32)] = 1.0
+    for k0 in range(0, K, M):
+        rows = min(M, K - k0)
+        eye = np.zeros((M, K), dtype=np.float32)
+        eye[np.arange(rows), k0 + np.arange(rows)] = 1.0
         x = torch.from_numpy(eye).to(torch.bfloat16).cuda()
         y = oracle.bf16_to_f64(from_dev_bf16(w3a16_gemm(x, packed, scales)))
-        want = w[:, k0:k0 + 32].T.astype(np.float64)
-        assert np.all(np.abs(y - want) <= 2.0 ** -8 * np.abs(want) + 1e-30), k0
+        want = w[:, k0:k0 + rows].T.astype(np.float64)
+        got = y[:rows]
+        assert np.all(np.abs(got - want) <= 2.0 ** -8 * np.abs(want) + 1e-30), (M, N, K, k0)
+        assert np.all(y[rows:] == 0.0), (M, N, K, k0)  # rows of x that are zero give zero
+    w3_check_device_error()
 
 
-def test_position_probe(orc):
-    # x = e_k picks column k of W: the result is one dequantized weight, rounded once
-    N, K = 40, 256
-    p = make_problem(16, N, K, seed=15)
-    _, codes, scales = device_problem(p)
-    packed = w3_pack(codes)
-    w = orc.dequant_f32(orc.pack(p.codes), p.scales_bf16, K)
-    for k0 in range(0, K, 16):
-        eye = np.zeros((16, K), dtype=np.float32)
-        eye[np.arange(16), k0 + np.arange(16)] = 1.0
-        x = torch.from_numpy(eye).to(torch.bfloat16).cuda()
-        y = oracle.bf16_to_f64(from_dev_bf16(w3a16_gemm(x, packed, scales)))
-        want = w[:, k0:k0 + 16].T.astype(np.float64)
-        assert np.all(np.abs(y - want) <= 2.0 ** -8 * np.abs(want) + 1e-30), k0
+# (route, M, N, K): one probe shape per kernel route; the route is asserted first
+PROBES = [
+    ("decode_sk", 1, 4800, 256),
+    ("decode_sk", 4, 4800, 384),
+    ("decode", 16, 40, 256),
+    ("decode", 1, 300, 256),
+    ("decode_tc", 8, 300, 256),
+    ("decode_tc", 16, 512, 384),
+    ("decode_tc32", 32, 300, 512),
+    ("prefill", 64, 300, 256),
+    ("prefill_ab", 256, 1024, 1024),
+    ("passes", 40, 300, 128),
+]
+
+
+@pytest.mark.parametrize("route,M,N,K", PROBES, ids=[f"{r}_M{m}_N{n}_K{k}" for r, m, n, k in PROBES])
+def test_position_probe(orc, route, M, N, K):
+    assert w3a16_gemm_route(M, N, K) == route
+    _probe(orc, M, N, K, seed=15)
 
 
 def test_row_concatenated_weights_are_one_weight(orc):
@@ -186,8 +203,7 @@ def test_row_concatenated_weights_are_one_weight(orc):
         n0 += p.N
 
 
-def _sampled_check(orc, name, n_samples=1024, seed=0):
-    wl = workloads()[name]
+def _device_run(orc, wl):
     p = wl.problem()
     x, codes, scales = device_problem(p)
     packed = w3_pack(codes)
@@ -196,32 +212,48 @@ def _sampled_check(orc, name, n_samples=1024, seed=0):
     del codes
     y = from_dev_bf16(w3a16_gemm(x, packed, scales))
     w3_check_device_error()
-    rng = np.random.Generator(np.random.PCG64(seed))
-    ms = rng.integers(0, wl.M, n_samples)
-    ns = rng.integers(0, wl.N, n_samples)
-    # always include the corners and the last row/column
-    ms = np.concatenate([ms, [0, wl.M - 1, 0, wl.M - 1]])
-    ns = np.concatenate([ns, [0, 0, wl.N - 1, wl.N - 1]])
-    ref = orc.gemm_f64_entries(p.x_bf16, ref_packed, p.scales_bf16, ms, ns)
-    norms = orc.weight_row_norms(ref_packed[ns], p.scales_bf16[ns], wl.K)
-    xf = oracle.bf16_to_f64(p.x_bf16[ms])
-    tol = 1e-2 * np.sqrt(np.sum(xf * xf, axis=1)) * norms / np.sqrt(wl.K) + 1e-3
-    worst = assert_within_bound(y[ms, ns][None, :], ref[None, :], tol[None, :], name)
-    print(f"{name}: worst |err|/bound = {worst:.3g} over {ms.size} sampled outputs")
+    return p, ref_packed, y
 
 
 FULL = [n for n in workloads() if not n.startswith("prefill")]
 
 
 @pytest.mark.parametrize("name", FULL)
-def test_full_size_sampled(orc, name):
-    _sampled_check(orc, name)
+def test_full_size_full_parity(orc, name):
+    """Every output of the full-size decode workload against the fp64 oracle (all cores)."""
+    wl = workloads()[name]
+    p, ref_packed, y = _device_run(orc, wl)
+    ref = orc.gemm_f64(p.x_bf16, ref_packed, p.scales_bf16, threads=0)
+    tol = bound(p.x_bf16, orc.weight_row_norms(ref_packed, p.scales_bf16, wl.K), wl.K)
+    worst = assert_within_bound(y, ref, tol, name)
+    print(f"{name} ({w3a16_gemm_route(wl.M, wl.N, wl.K)}): worst |err|/bound = {worst:.3g} over {y.size} outputs")
 
 
-def test_prefill_full_size_sampled(orc):
-    _sampled_check(orc, "prefill_2048x28672x8192", n_samples=4096)
+def _rows_and_entries_check(orc, name, n_rows=64, n_samples=4096, seed=0):
+    """64 random whole rows of y (every n) plus 4096 random (m, n) entries against the oracle."""
+    wl = workloads()[name]
+    p, ref_packed, y = _device_run(orc, wl)
+    rng = np.random.Generator(np.random.PCG64(seed))
+    rows = np.sort(rng.choice(wl.M, size=n_rows, replace=False))
+    rows[-1] = wl.M - 1  # always the last row
+    norms = orc.weight_row_norms(ref_packed, p.scales_bf16, wl.K)
+    ref_rows = orc.gemm_f64(p.x_bf16[rows], ref_packed, p.scales_bf16, threads=0)
+    worst = assert_within_bound(y[rows], ref_rows, bound(p.x_bf16[rows], norms, wl.K), f"{name} rows")
+    ms = np.concatenate([rng.integers(0, wl.M, n_samples), [0, wl.M - 1, 0, wl.M - 1]])
+    ns = np.concatenate([rng.integers(0, wl.N, n_samples), [0, 0, wl.N - 1, wl.N - 1]])
+    ref = orc.gemm_f64_entries(p.x_bf16, ref_packed, p.scales_bf16, ms, ns)
+    xf = oracle.bf16_to_f64(p.x_bf16[ms])
+    tol = 1e-2 * np.sqrt(np.sum(xf * xf, axis=1)) * norms[ns] / np.sqrt(wl.K) + 1e-3
+    worst = max(worst, assert_within_bound(y[ms, ns][None, :], ref[None, :], tol[None, :], name))
+    print(f"{name} ({w3a16_gemm_route(wl.M, wl.N, wl.K)}): worst |err|/bound = {worst:.3g} over {n_rows} rows "
+          f"and {ms.size} entries")
 
 
-def test_prefill_tensor_memory_kernel_full_size_sampled(orc):
+def test_prefill_full_size_rows_and_entries(orc):
+    _rows_and_entries_check(orc, "prefill_2048x28672x8192")
+
+
+def test_prefill_tensor_memory_kernel_full_size_rows_and_entries(orc):
     # M = 1024 on gate_proj: the weights-in-tensor-memory prefill kernel is the one launched
-    _sampled_check(orc, "prefill_1024x28672x8192", n_samples=4096)
+    assert w3a16_gemm_route(1024, 28672, 8192) == "prefill_ab"
+    _rows_and_entries_check(orc, "prefill_1024x28672x8192")

@@ -21,7 +21,7 @@ MUTANTS = [
     ("word_bits_msb_first_both_sides",
      "(row[b / 32] >> (b % 32)) & 1u", "(row[b / 32] >> (31 - b % 32)) & 1u", 1),
     ("group_index_reversed", "scales[n * G + k / ORACLE_GROUP]", "scales[n * G + (K - 1 - k) / ORACLE_GROUP]", 2),
-    ("output_transposed", "y[m * N + n] = dot_row", "y[n * M + m] = dot_row", 1),
+    ("output_transposed", "y[m * N + n] = dot_row", "y[n * M + m] = dot_row", 2),
     ("dropped_last_term", "for (int64_t k = 0; k < K; ++k)\n        acc +=", "for (int64_t k = 0; k < K - 1; ++k)\n        acc +=", 1),
     ("x_reversed_along_k", "x[m * K + k]", "x[m * K + (K - 1 - k)]", 1),
     ("sign_flipped", "(int)code_at(row, k) - 4", "4 - (int)code_at(row, k)", 2),

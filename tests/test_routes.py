@@ -1,0 +1,65 @@
+"""Kernel selection of w3a16_gemm, asked through the C ABI without a GPU.
+
+w3a16_gemm_route depends only on the shape and the SM count, so the dispatch
+rules can be checked on the host: which kernel serves each batch size of the
+benchmarked shapes, the batch-size boundaries between routes, and that invalid
+shapes have no route.
+"""
+import pytest
+
+from w3a16_gemv_b200 import _binding, build, w3a16_gemm_route
+
+SMS = 148  # B200
+
+ROUTES = {"decode_sk", "decode", "decode_tc", "decode_tc32", "prefill", "prefill_ab", "passes"}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def lib():
+    build.build()
+    return _binding.lib()
+
+
+def test_invalid_shapes_have_no_route(lib):
+    f = lib.w3a16_gemm_route
+    assert f(0, 16, 128, SMS) is None
+    assert f(1, 0, 128, SMS) is None
+    assert f(1, 16, 192, SMS) is None
+    assert f(1, 16, 0, SMS) is None
+    assert f(1, 16, 128, 0) is None
+
+
+@pytest.mark.parametrize("M", list(range(1, 70)) + [128, 255, 256, 257, 1024, 2048, 4096])
+@pytest.mark.parametrize("N,K", [(28672, 8192), (8192, 28672), (8192, 8192), (1024, 8192), (4096, 4096),
+                                 (300, 1152), (40, 256), (28672, 128)])
+def test_every_shape_has_a_known_route(M, N, K):
+    r = w3a16_gemm_route(M, N, K, num_sms=SMS)
+    assert r in ROUTES
+    if M <= 16:
+        assert r in ("decode_sk", "decode", "decode_tc")
+    if r == "decode_sk":
+        assert M <= 4 and N >= 32 * SMS
+    if r in ("decode_tc", "decode_tc32"):
+        assert N >= 256
+    if r == "decode_tc32":
+        assert 17 <= M <= 32
+    if r in ("prefill", "prefill_ab"):
+        assert M > 16 and K >= 256
+    if r == "passes":
+        assert M > 16 and K < 256
+
+
+def test_benchmarked_shapes():
+    # the gate_proj decode step M = 1, 4, 16 and the M = 2048 prefill
+    assert w3a16_gemm_route(1, 28672, 8192, SMS) == "decode_sk"
+    assert w3a16_gemm_route(4, 28672, 8192, SMS) == "decode_sk"
+    assert w3a16_gemm_route(16, 28672, 8192, SMS) == "decode_tc"
+    assert w3a16_gemm_route(2048, 28672, 8192, SMS) in ("prefill", "prefill_ab")
+    # fewer 32-row blocks than SMs: not the stream-K decode
+    assert w3a16_gemm_route(1, 1024, 8192, SMS) == "decode"
+
+
+def test_route_depends_on_the_sm_count():
+    # the stream-K decode needs one 32-row block per SM
+    assert w3a16_gemm_route(1, 4800, 1024, 148) == "decode_sk"
+    assert w3a16_gemm_route(1, 4800, 1024, 160) == "decode"

@@ -21,6 +21,7 @@ from ._binding import (  # noqa: F401
     w3_unpack,
     w3a16_gemm,
     w3a16_gemm_noalloc,
+    w3a16_gemm_route,
 )
 
 __all__ = [
@@ -36,4 +37,5 @@ __all__ = [
     "w3_unpack",
     "w3a16_gemm",
     "w3a16_gemm_noalloc",
+    "w3a16_gemm_route",
 ]

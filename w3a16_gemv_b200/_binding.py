@@ -43,6 +43,7 @@ SIGNATURES = [
     ("w3_repack_ct4", ctypes.c_int, [_P, _P, _I64, _I64, _P, _P]),
     ("w3a16_gemm", ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P]),
     ("w3a16_gemm_noalloc", ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P]),
+    ("w3a16_gemm_route", ctypes.c_char_p, [_I64, _I64, _I64, ctypes.c_int32]),
     ("w3_check_device_error", ctypes.c_int, [_P]),
 ]
 
@@ -199,6 +200,17 @@ def _gemm(entry: str, x: torch.Tensor, packed: torch.Tensor, scales: torch.Tenso
     _check(getattr(lib(), entry)(x.data_ptr(), packed.data_ptr(), scales.data_ptr(), out.data_ptr(), M, N, K,
                                  _stream(stream)), entry)
     return out
+
+
+def w3a16_gemm_route(M: int, N: int, K: int, num_sms: int | None = None) -> str:
+    """The kernel route w3a16_gemm takes for M x N x K (see include/w3a16.h).  num_sms defaults to
+    the current CUDA device's SM count; pass it explicitly to ask without a GPU."""
+    if num_sms is None:
+        num_sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    r = lib().w3a16_gemm_route(M, N, K, num_sms)
+    if r is None:
+        raise ValueError(f"w3a16_gemm_route: no route for M={M} N={N} K={K} num_sms={num_sms}")
+    return r.decode()
 
 
 def w3_check_device_error(stream=None) -> None:

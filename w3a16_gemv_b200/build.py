@@ -32,21 +32,22 @@ def nvcc() -> str:
     raise RuntimeError("nvcc not found: the CUDA toolkit is needed to build libw3a16.so")
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(path: str = LIB) -> bool:
+    if not os.path.exists(path):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(path)
     return all(os.path.getmtime(s) <= t for s in sources())
 
 
 def build(force: bool = False, verbose: bool = False, out: str | None = None, defines=()) -> str:
     """Compile the library if it is missing or older than its sources; return its path.
 
-    `out` and `defines` (e.g. ``["W3_DECODE_DEPTH=3"]``) build a variant elsewhere,
-    for tuning sweeps; the default build uses the constants in the sources."""
+    `out` and `defines` build a variant of the library elsewhere: the failure-detection
+    test builds one with ``W3_TEST_HOOKS`` (a test-only kernel that makes a bounded wait run
+    out) and a short ``W3_WAIT_LIMIT_CYCLES``.  The product build has neither."""
     target = out or LIB
-    if not force and out is None and up_to_date():
-        return LIB
+    if not force and up_to_date(target):
+        return target
     tmp = target + f".tmp{os.getpid()}"
     cmd = [nvcc(), *ARCH_FLAGS, *NVCC_FLAGS, *[f"-D{d}" for d in defines], "-o", tmp,
            os.path.join(CSRC, "api.cu")]

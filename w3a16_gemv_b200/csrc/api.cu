@@ -26,28 +26,6 @@
 #include "prefill_gemm.cuh"
 #include "prefill_swab.cuh"
 
-#ifndef W3_DECODE_TMA2D
-#define W3_DECODE_TMA2D 1
-#endif
-#ifndef W3_DECODE_STREAMK
-#define W3_DECODE_STREAMK 1
-#endif
-#ifndef W3_PREFILL_TCGEN05
-#define W3_PREFILL_TCGEN05 1
-#endif
-// Smallest decode batch that uses the tcgen05 decode kernel (above 16: never).
-// Launch the decode kernels with programmatic dependent launch.
-#ifndef W3_DECODE_PDL
-#define W3_DECODE_PDL 1
-#endif
-// The prefill with the weights in tensor memory (prefill_swab.cuh): a candidate for M >= 256.
-#ifndef W3_PREFILL_SWAB
-#define W3_PREFILL_SWAB 1
-#endif
-#ifndef W3_DECODE_TC_MIN_M
-#define W3_DECODE_TC_MIN_M 5
-#endif
-
 namespace w3 {
 namespace {
 
@@ -224,7 +202,7 @@ w3_status launch_decode_sk(const uint16_t *x, const int32_t *packed, const uint1
     cudaLaunchAttribute attr[1];
     set_pdl(attr[0]);  // overlaps the set-up with the previous kernel's tail
     cfg.attrs = attr;
-    cfg.numAttrs = W3_DECODE_PDL ? 1 : 0;
+    cfg.numAttrs = 1;
     cudaError_t e;
     switch (P.mt) {
         case 1: e = cudaLaunchKernelEx(&cfg, decode_sk::decode_sk_kernel<1>, prm); break;
@@ -278,7 +256,7 @@ w3_status launch_decode_tc(const uint16_t *x, const int32_t *packed, const uint1
     cudaLaunchAttribute mattr[1];
     set_pdl(mattr[0]);
     cfg.attrs = mattr;
-    cfg.numAttrs = W3_DECODE_PDL ? 1 : 0;
+    cfg.numAttrs = 1;
     if (I::launch(cfg, prm) != cudaSuccess) return W3_ERR_CUDA;
     if (P.P == 1) return W3_OK;
     typename I::FixupT fp;
@@ -401,7 +379,7 @@ w3_status launch_decode(const uint16_t *x, const int32_t *packed, const uint16_t
     // one tiled TMA copy per stage when the box fits inside the matrix, else per-row bulk copies
     prm.use_tma2d = 0;
     const int64_t words = static_cast<int64_t>(K) * 3 / 32;
-    if (W3_DECODE_TMA2D && N >= decode::kRowsPerWarp && words >= decode::kRowPitchWords) {
+    if (N >= decode::kRowsPerWarp && words >= decode::kRowPitchWords) {
         PFN_cuTensorMapEncodeTiled enc = tensor_map_encoder();
         if (!enc) return W3_ERR_CUDA;
         cuuint64_t dims[2] = {static_cast<cuuint64_t>(words), static_cast<cuuint64_t>(N)};
@@ -440,6 +418,52 @@ w3_status launch_decode(const uint16_t *x, const int32_t *packed, const uint16_t
     return e == cudaSuccess ? W3_OK : W3_ERR_CUDA;
 }
 
+// ---- kernel selection (host logic only: depends on the shape and the SM count) --------
+
+// Smallest batch that runs on the tensor-core decode (below it the mma.sync decodes).
+constexpr int kTcMinBatch = 5;
+
+enum class Route {
+    DecodeStreamK,  // decode_sk_kernel: M <= 4, at least one 32-row block per SM
+    Decode,         // decode_kernel: the remaining small shapes (M <= 16)
+    DecodeTc,       // decode_tc_kernel (+ fix-up): 5 <= M <= 16, N >= 256
+    DecodeTc32,     // decode_tc32 decode_tc_kernel (+ fix-up): 17 <= M <= 32, N >= 256
+    Prefill,        // prefill_kernel: M > 16 (not on the 32-wide decode), K >= 256
+    PrefillAb,      // prefill_ab_kernel: chosen over prefill_kernel per shape
+    Passes,         // no prefill kernel fits (K < 256): 16-row passes of the decode routes
+};
+
+// The route of one pass of at most 16 batch rows.
+Route decode_route(int64_t mb, int64_t N, int64_t K, int sms) {
+    if (N >= decode_tc::kRows && mb >= kTcMinBatch) return Route::DecodeTc;
+    if (N >= static_cast<int64_t>(decode_sk::kBlockRows) * sms &&
+        decode_sk::applicable(static_cast<int>(mb), static_cast<int>(N), static_cast<int>(K)))
+        return Route::DecodeStreamK;
+    return Route::Decode;
+}
+
+Route choose_route(int64_t M, int64_t N, int64_t K, int sms) {
+    if (M <= 16) return decode_route(M, N, K, sms);
+    if (M <= decode_tc32::kBatch && N >= decode_tc32::kRows) return Route::DecodeTc32;
+    // the prefill kernels' packed-word copies are 24 words wide: rows of at least 256 codes
+    if (K >= 256)
+        return prefer_prefill_ab(static_cast<int>(M), static_cast<int>(N), sms) ? Route::PrefillAb : Route::Prefill;
+    return Route::Passes;
+}
+
+const char *route_name(Route r) {
+    switch (r) {
+        case Route::DecodeStreamK: return "decode_sk";
+        case Route::Decode: return "decode";
+        case Route::DecodeTc: return "decode_tc";
+        case Route::DecodeTc32: return "decode_tc32";
+        case Route::Prefill: return "prefill";
+        case Route::PrefillAb: return "prefill_ab";
+        case Route::Passes: return "passes";
+    }
+    return "";
+}
+
 // Fixed scratch of w3a16_gemm_noalloc: the fp32 partial sums of the tensor-core
 // decode for up to kNoAllocMaxCtas CTAs (one per SM).  Every slot the fix-up
 // kernel reads is written by the main kernel of the same call, so nothing in
@@ -466,6 +490,106 @@ float *noalloc_scratch() {
     });
     return st.scratch;
 }
+
+// Where the tensor-core decode keeps its partial sums: a stream-ordered allocation
+// from `pool` (w3a16_gemm), or the fixed array `fixed` of `fixed_floats` floats
+// (w3a16_gemm_noalloc, which must never allocate).
+struct ScratchSource {
+    cudaMemPool_t pool = nullptr;
+    float *fixed = nullptr;
+    int64_t fixed_floats = 0;
+
+    w3_status acquire(int64_t floats, cudaStream_t st, float **out) const {
+        *out = nullptr;
+        if (floats <= 0) return W3_OK;
+        if (!pool) {
+            if (!fixed) return W3_ERR_CUDA;
+            if (floats > fixed_floats) return W3_ERR_UNSUPPORTED;
+            *out = fixed;
+            return W3_OK;
+        }
+        return cudaMallocFromPoolAsync(reinterpret_cast<void **>(out), floats * sizeof(float), pool, st) ==
+                       cudaSuccess
+                   ? W3_OK
+                   : W3_ERR_CUDA;
+    }
+    w3_status release(float *p, cudaStream_t st) const {
+        if (!p || !pool) return W3_OK;
+        return cudaFreeAsync(p, st) == cudaSuccess ? W3_OK : W3_ERR_CUDA;
+    }
+};
+
+// y = x W^T for validated arguments: the route's kernels, in stream order.
+w3_status run_gemm(const uint16_t *x, const int32_t *packed, const uint16_t *scales, uint16_t *y, int64_t M,
+                   int64_t N, int64_t K, int sms, cudaStream_t st, const ScratchSource &scratch) {
+    const int n = static_cast<int>(N), k = static_cast<int>(K);
+    const Route route = choose_route(M, N, K, sms);
+    if (route == Route::Prefill) return launch_prefill(x, packed, scales, y, static_cast<int>(M), n, k, sms, st);
+    if (route == Route::PrefillAb) return launch_prefill_ab(x, packed, scales, y, static_cast<int>(M), n, k, st);
+    if (route == Route::DecodeTc32) {
+        const decode_tc32::LaunchPlan plan32 = decode_tc32::plan(N, K, sms);
+        float *partial = nullptr;
+        if (w3_status s = scratch.acquire(plan32.ws_floats, st, &partial)) return s;
+        w3_status status = launch_decode_tc<decode_tc32::Instance>(x, packed, scales, y, static_cast<int>(M), n, k,
+                                                                   plan32, partial, st);
+        if (w3_status s = scratch.release(partial, st); s && status == W3_OK) status = s;
+        return status;
+    }
+    // Decode routes, in passes of at most 16 batch rows (one pass unless M > 16 with K < 256,
+    // where no prefill kernel fits); the tensor-core passes share one scratch buffer.
+    const decode_tc::LaunchPlan tplan = decode_tc::plan(N, K, sms);
+    bool any_tc = false;
+    for (int64_t m0 = 0; m0 < M; m0 += 16)
+        any_tc = any_tc || decode_route(std::min<int64_t>(16, M - m0), N, K, sms) == Route::DecodeTc;
+    float *partial = nullptr;
+    if (any_tc) {
+        if (w3_status s = scratch.acquire(tplan.ws_floats, st, &partial)) return s;
+    }
+    w3_status status = W3_OK;
+    for (int64_t m0 = 0; m0 < M && status == W3_OK; m0 += 16) {
+        const int mb = static_cast<int>(std::min<int64_t>(16, M - m0));
+        const uint16_t *xp = x + m0 * K;
+        uint16_t *yp = y + m0 * N;
+        switch (decode_route(mb, N, K, sms)) {
+            case Route::DecodeTc:
+                status = launch_decode_tc<decode_tc::Instance>(xp, packed, scales, yp, mb, n, k, tplan, partial, st);
+                break;
+            case Route::DecodeStreamK: status = launch_decode_sk(xp, packed, scales, yp, mb, n, k, sms, st); break;
+            default: status = launch_decode(xp, packed, scales, yp, mb, n, k, sms, st); break;
+        }
+    }
+    if (w3_status s = scratch.release(partial, st); s && status == W3_OK) status = s;
+    return status;
+}
+
+// The checks every product entry point makes before anything is launched.
+w3_status check_gemm_args(const uint16_t *x, const int32_t *packed, const uint16_t *scales, const uint16_t *y,
+                          int64_t M, int64_t N, int64_t K) {
+    if (!x || !packed || !scales || !y) return W3_ERR_NULL;
+    if (w3_status s = check_nk(N, K)) return s;
+    if (M < 1 || M > kMaxDim || M * K > kMaxElems || M * N > kMaxElems) return W3_ERR_SHAPE;
+    if (!aligned16(x) || !aligned16(packed) || !aligned16(scales) || !aligned16(y)) return W3_ERR_ALIGN;
+    const int64_t ybytes = M * N * 2;
+    if (overlaps(y, ybytes, x, M * K * 2) || overlaps(y, ybytes, packed, N * K * 3 / 8) ||
+        overlaps(y, ybytes, scales, N * (K / kGroup) * 2))
+        return W3_ERR_ALIAS;
+    return W3_OK;
+}
+
+#ifdef W3_TEST_HOOKS
+// Test-only: one thread waits, with the bounded wait every kernel uses, on an
+// mbarrier phase that nothing completes, so the wait runs out and records the
+// timeout flag.  Built only into the test variant of the library (which also
+// shortens the wait limit).
+__global__ void wait_timeout_kernel() {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_addr(&bar), 1);
+        mbar_init_fence();
+        (void)mbar_wait_bounded(smem_addr(&bar), 0);
+    }
+}
+#endif
 
 }  // namespace
 }  // namespace w3
@@ -559,102 +683,40 @@ w3_status w3_dequant_f32(const int32_t *packed, const uint16_t *scales, float *w
 
 w3_status w3a16_gemm(const uint16_t *x, const int32_t *packed, const uint16_t *scales, uint16_t *y, int64_t M,
                      int64_t N, int64_t K, w3_stream_t stream) {
-    if (!x || !packed || !scales || !y) return W3_ERR_NULL;
-    if (w3_status s = check_nk(N, K)) return s;
-    if (M < 1 || M > kMaxDim || M * K > kMaxElems || M * N > kMaxElems) return W3_ERR_SHAPE;
-    if (!aligned16(x) || !aligned16(packed) || !aligned16(scales) || !aligned16(y)) return W3_ERR_ALIGN;
-    const int64_t ybytes = M * N * 2;
-    if (overlaps(y, ybytes, x, M * K * 2) || overlaps(y, ybytes, packed, N * K * 3 / 8) ||
-        overlaps(y, ybytes, scales, N * (K / kGroup) * 2))
-        return W3_ERR_ALIAS;
+    if (w3_status s = check_gemm_args(x, packed, scales, y, M, N, K)) return s;
     int sms;
     cudaMemPool_t pool;
     if (w3_status s = device_setup(&sms, &pool)) return s;
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    // 17 <= M <= 32: the 32-wide tensor-core decode (N >= 256)
-    if (M > 16 && M <= decode_tc32::kBatch && N >= decode_tc32::kRows) {
-        const decode_tc32::LaunchPlan plan32 = decode_tc32::plan(N, K, sms);
-        float *partial = nullptr;
-        if (plan32.ws_floats > 0 &&
-            cudaMallocFromPoolAsync(reinterpret_cast<void **>(&partial), plan32.ws_floats * sizeof(float), pool, st) !=
-                cudaSuccess)
-            return W3_ERR_CUDA;
-        w3_status status = launch_decode_tc<decode_tc32::Instance>(x, packed, scales, y, static_cast<int>(M),
-                                                                   static_cast<int>(N), static_cast<int>(K), plan32,
-                                                                   partial, st);
-        if (partial && cudaFreeAsync(partial, st) != cudaSuccess && status == W3_OK) status = W3_ERR_CUDA;
-        return status;
-    }
-    // the prefill kernels' packed-word copies are 24 words wide: rows of at least 256 codes
-    if (M > 16 && W3_PREFILL_TCGEN05 && K >= 256) {
-        if (W3_PREFILL_SWAB && prefer_prefill_ab(static_cast<int>(M), static_cast<int>(N), sms))
-            return launch_prefill_ab(x, packed, scales, y, static_cast<int>(M), static_cast<int>(N),
-                                     static_cast<int>(K), st);
-        return launch_prefill(x, packed, scales, y, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), sms,
-                              st);
-    }
-    // The tensor-core decode for N >= 256: one call per 16 batch rows, all sharing
-    // one stream-ordered scratch buffer for the partial sums.
-    const bool tc = N >= decode_tc::kRows && W3_DECODE_TC_MIN_M <= std::min<int64_t>(M, 16);
-    const decode_tc::LaunchPlan tplan = decode_tc::plan(N, K, sms);
-    float *partial = nullptr;
-    if (tc && tplan.ws_floats > 0 &&
-        cudaMallocFromPoolAsync(reinterpret_cast<void **>(&partial), tplan.ws_floats * sizeof(float), pool, st) !=
-            cudaSuccess)
-        return W3_ERR_CUDA;
-    w3_status status = W3_OK;
-    // Batches above 16 rows without the tensor-core path run as 16-row decode passes.
-    for (int64_t m0 = 0; m0 < M && status == W3_OK; m0 += 16) {
-        const int mb = static_cast<int>(std::min<int64_t>(16, M - m0));
-        if (tc && mb >= W3_DECODE_TC_MIN_M) {
-            status = launch_decode_tc<decode_tc::Instance>(x + m0 * K, packed, scales, y + m0 * N, mb,
-                                                           static_cast<int>(N), static_cast<int>(K), tplan, partial, st);
-            if (status == W3_OK) continue;
-            if (status != W3_ERR_UNSUPPORTED) break;
-            status = W3_OK;
-        }
-        // fewer 32-row blocks than SMs: the cluster split-K decode spreads K over more SMs
-        const bool sk = W3_DECODE_STREAMK && N >= static_cast<int64_t>(decode_sk::kBlockRows) * sms &&
-                        decode_sk::applicable(mb, static_cast<int>(N), static_cast<int>(K));
-        status = sk ? launch_decode_sk(x + m0 * K, packed, scales, y + m0 * N, mb, static_cast<int>(N),
-                                       static_cast<int>(K), sms, st)
-                    : launch_decode(x + m0 * K, packed, scales, y + m0 * N, mb, static_cast<int>(N),
-                                    static_cast<int>(K), sms, st);
-    }
-    if (partial && cudaFreeAsync(partial, st) != cudaSuccess && status == W3_OK) status = W3_ERR_CUDA;
-    return status;
+    ScratchSource scratch;
+    scratch.pool = pool;
+    return run_gemm(x, packed, scales, y, M, N, K, sms, reinterpret_cast<cudaStream_t>(stream), scratch);
 }
 
 w3_status w3a16_gemm_noalloc(const uint16_t *x, const int32_t *packed, const uint16_t *scales, uint16_t *y,
                              int64_t M, int64_t N, int64_t K, w3_stream_t stream) {
-    if (!x || !packed || !scales || !y) return W3_ERR_NULL;
-    if (w3_status s = check_nk(N, K)) return s;
-    if (M < 1 || M > kMaxDim || M * K > kMaxElems || M * N > kMaxElems) return W3_ERR_SHAPE;
-    if (!aligned16(x) || !aligned16(packed) || !aligned16(scales) || !aligned16(y)) return W3_ERR_ALIGN;
-    const int64_t ybytes = M * N * 2;
-    if (overlaps(y, ybytes, x, M * K * 2) || overlaps(y, ybytes, packed, N * K * 3 / 8) ||
-        overlaps(y, ybytes, scales, N * (K / kGroup) * 2))
-        return W3_ERR_ALIAS;
+    if (w3_status s = check_gemm_args(x, packed, scales, y, M, N, K)) return s;
     int sms;
     if (w3_status s = device_setup(&sms)) return s;
-    // Only the tensor-core decode (W3_DECODE_TC_MIN_M <= M <= 32, N >= 256) uses
-    // scratch; every other shape takes w3a16_gemm's path, which allocates nothing.
-    if (M > decode_tc32::kBatch || M < W3_DECODE_TC_MIN_M || N < decode_tc::kRows)
-        return w3a16_gemm(x, packed, scales, y, M, N, K, stream);
-    float *scratch = noalloc_scratch();
-    if (!scratch) return W3_ERR_CUDA;
-    const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (M > decode_tc::kBatch) {
-        const decode_tc32::LaunchPlan plan32 = decode_tc32::plan(N, K, sms);
-        if (plan32.ws_floats > kNoAllocScratchFloats) return W3_ERR_UNSUPPORTED;
-        return launch_decode_tc<decode_tc32::Instance>(x, packed, scales, y, static_cast<int>(M), static_cast<int>(N),
-                                                       static_cast<int>(K), plan32, scratch, st);
-    }
-    const decode_tc::LaunchPlan tplan = decode_tc::plan(N, K, sms);
-    if (tplan.ws_floats > kNoAllocScratchFloats) return W3_ERR_UNSUPPORTED;
-    return launch_decode_tc<decode_tc::Instance>(x, packed, scales, y, static_cast<int>(M), static_cast<int>(N),
-                                                 static_cast<int>(K), tplan, scratch, st);
+    ScratchSource scratch;  // no pool: every route that needs scratch gets the fixed array
+    scratch.fixed = noalloc_scratch();
+    scratch.fixed_floats = kNoAllocScratchFloats;
+    if (!scratch.fixed) return W3_ERR_CUDA;
+    return run_gemm(x, packed, scales, y, M, N, K, sms, reinterpret_cast<cudaStream_t>(stream), scratch);
 }
+
+const char *w3a16_gemm_route(int64_t M, int64_t N, int64_t K, int32_t num_sms) {
+    if (M < 1 || check_nk(N, K) != W3_OK || M > kMaxDim || num_sms < 1) return nullptr;
+    return route_name(choose_route(M, N, K, num_sms));
+}
+
+#ifdef W3_TEST_HOOKS
+w3_status w3_test_wait_timeout(w3_stream_t stream) {
+    int sms;
+    if (w3_status s = device_setup(&sms)) return s;
+    wait_timeout_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>();
+    return launch_status();
+}
+#endif
 
 w3_status w3_check_device_error(w3_stream_t stream) {
     if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return W3_ERR_CUDA;

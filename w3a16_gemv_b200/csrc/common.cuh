@@ -26,7 +26,11 @@ constexpr unsigned kDevErrTimeout = 1u;
 // A bounded wait gives up after this many SM clock cycles (about 2 s at the
 // B200's 1.965 GHz maximum; the SM cycle counter is cheap to read, unlike the
 // global timer).
-constexpr long long kWaitLimitCycles = 4000000000ll;
+// (The test variant of the library shortens it to make a wait run out quickly.)
+#ifndef W3_WAIT_LIMIT_CYCLES
+#define W3_WAIT_LIMIT_CYCLES 4000000000ll
+#endif
+constexpr long long kWaitLimitCycles = W3_WAIT_LIMIT_CYCLES;
 
 // Set by kernels, read and cleared by w3_check_device_error (the library is one
 // translation unit, so this is its only definition).
@@ -63,15 +67,6 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
 
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
-#if defined(W3_WAIT_TEST)
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-#else
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
@@ -79,7 +74,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         : "=r"(ok)
         : "r"(bar), "r"(parity)
         : "memory");
-#endif
     return ok != 0;
 }
 
