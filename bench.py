@@ -46,6 +46,7 @@ ROTATE = 5
 WORKLOAD = "Llama-3.1-70B gate_proj N=28672 K=8192, W3A16 g128 decode batch M=1,4,16"
 FALLBACK_HBM_GBS = 6650.0
 DECODE_SOURCES = ("w3a16_gemv_b200/csrc/api.cu", "w3a16_gemv_b200/csrc/decode_gemv.cuh",
+                  "w3a16_gemv_b200/csrc/decode_split.cuh",
                   "w3a16_gemv_b200/csrc/decode_streamk.cuh", "w3a16_gemv_b200/csrc/decode_tcgen05.cuh",
                   "w3a16_gemv_b200/csrc/prefill_gemm.cuh", "w3a16_gemv_b200/csrc/common.cuh")
 
@@ -56,6 +57,7 @@ def algorithmic_bytes(M: int, N: int, K: int) -> int:
 
 # kernel symbol of each route of w3a16_gemm_route (the names in an ncu launch list)
 ROUTE_KERNELS = {
+    "decode_split": "w3::dsplit::decode_split_kernel",
     "decode_sk": "w3::decode_sk::decode_sk_kernel",
     "decode": "w3::decode::decode_kernel",
     "decode_tc": "w3::decode_tc::decode_tc_kernel",

@@ -50,13 +50,14 @@ SMALL = [
     (13, 28672, 256, "uniform8", "lognormal", "normal"),          # many row tiles, two groups
     (1, 2000, 128, "uniform8", "lognormal", "normal"),
     (1, 64, 28672, "gsq_5level", "absnormal", "normal_outliers"),
-    # the stream-K decode (M <= 4 with at least as many 32-row blocks as SMs): ragged blocks,
-    # odd group counts, blocks split between warps
+    # many 32-row blocks: ragged last block, odd group counts, blocks split between warps and
+    # K split over thread-block clusters
     (1, 4800, 384, "uniform8", "lognormal", "normal"),
     (3, 5000, 1152, "gsq_5level", "absnormal", "normal_outliers"),
     (4, 6000, 640, "uniform8", "lognormal", "normal"),
     (2, 4736, 3968, "gsq_uniform", "lognormal", "normal"),
-    # a single group (K = 128) on every path: tcgen05 decode 16 and 32 wide, 16-row passes above 32
+    # a single group (K = 128) on every path: the split decode, the 32-wide tcgen05 decode, 16-row
+    # passes above 32
     (8, 512, 128, "uniform8", "lognormal", "normal"),
     (24, 512, 128, "uniform8", "lognormal", "normal"),
     (40, 300, 128, "gsq_5level", "absnormal", "normal"),
@@ -164,10 +165,13 @@ def _probe(orc, M, N, K, seed):
 PROBES = [
     ("decode_sk", 1, 4800, 256),
     ("decode_sk", 4, 4800, 384),
-    ("decode", 16, 40, 256),
     ("decode", 1, 300, 256),
-    ("decode_tc", 8, 300, 256),
-    ("decode_tc", 16, 512, 384),
+    ("decode", 16, 20, 256),
+    ("decode_split", 5, 300, 384),
+    ("decode_split", 8, 1000, 256),
+    ("decode_split", 12, 64, 1152),
+    ("decode_split", 16, 512, 384),
+    ("decode_split", 16, 40, 128),
     ("decode_tc32", 32, 300, 512),
     ("prefill", 64, 300, 256),
     ("prefill_ab", 256, 1024, 1024),

@@ -11,7 +11,7 @@ from w3a16_gemv_b200 import _binding, build, w3a16_gemm_route
 
 SMS = 148  # B200
 
-ROUTES = {"decode_sk", "decode", "decode_tc", "decode_tc32", "prefill", "prefill_ab", "passes"}
+ROUTES = {"decode_split", "decode_sk", "decode", "decode_tc", "decode_tc32", "prefill", "prefill_ab", "passes"}
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -35,8 +35,10 @@ def test_invalid_shapes_have_no_route(lib):
 def test_every_shape_has_a_known_route(M, N, K):
     r = w3a16_gemm_route(M, N, K, num_sms=SMS)
     assert r in ROUTES
-    if M <= 16:
-        assert r in ("decode_sk", "decode", "decode_tc")
+    if 5 <= M <= 16:
+        assert r == ("decode_split" if N >= 32 else "decode")
+    if M <= 4:
+        assert r in ("decode_sk", "decode")
     if r == "decode_sk":
         assert M <= 4 and N >= 32 * SMS
     if r in ("decode_tc", "decode_tc32"):
@@ -53,10 +55,12 @@ def test_benchmarked_shapes():
     # the gate_proj decode step M = 1, 4, 16 and the M = 2048 prefill
     assert w3a16_gemm_route(1, 28672, 8192, SMS) == "decode_sk"
     assert w3a16_gemm_route(4, 28672, 8192, SMS) == "decode_sk"
-    assert w3a16_gemm_route(16, 28672, 8192, SMS) == "decode_tc"
+    assert w3a16_gemm_route(16, 28672, 8192, SMS) == "decode_split"
+    assert w3a16_gemm_route(24, 28672, 8192, SMS) == "decode_tc32"
     assert w3a16_gemm_route(2048, 28672, 8192, SMS) in ("prefill", "prefill_ab")
-    # fewer 32-row blocks than SMs: not the stream-K decode
+    # fewer 32-row blocks than SMs at M <= 4: the mma.sync decode with cluster split-K
     assert w3a16_gemm_route(1, 1024, 8192, SMS) == "decode"
+    assert w3a16_gemm_route(8, 20, 8192, SMS) == "decode"
 
 
 def test_route_depends_on_the_sm_count():

@@ -48,8 +48,8 @@ def test_noalloc_matches_allocating_entry_twice(case):
 
 
 def test_noalloc_within_the_oracle_bound(orc):
-    M, N, K = 16, 1024, 8192  # every row tile shared between CTAs: the partial sums live in the scratch
-    assert w3a16_gemm_route(M, N, K) == "decode_tc"
+    M, N, K = 24, 1024, 8192  # every row tile shared between CTAs: the partial sums live in the scratch
+    assert w3a16_gemm_route(M, N, K) == "decode_tc32"
     p = make_problem(M, N, K, "gsq_5level", "absnormal", "normal_outliers", seed=22)
     x, codes, scales = device_problem(p)
     packed = w3_pack(codes)

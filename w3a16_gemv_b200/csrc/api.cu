@@ -14,6 +14,7 @@
 #include "../../include/w3a16.h"
 #include "common.cuh"
 #include "decode_gemv.cuh"
+#include "decode_split.cuh"
 #include "decode_streamk.cuh"
 // the tensor-core decode, once per batch width (16: M <= 16; 32: 17 <= M <= 32)
 #include "decode_tcgen05.cuh"
@@ -69,6 +70,20 @@ w3_status device_setup(int *num_sms, cudaMemPool_t *pool = nullptr) {
             reinterpret_cast<const void *>(decode::decode_kernel<8>),
             reinterpret_cast<const void *>(decode::decode_kernel<16>),
         };
+        const void *split_kernels[] = {
+            reinterpret_cast<const void *>(dsplit::decode_split_kernel<1>),
+            reinterpret_cast<const void *>(dsplit::decode_split_kernel<2>),
+            reinterpret_cast<const void *>(dsplit::decode_split_kernel<4>),
+            reinterpret_cast<const void *>(dsplit::decode_split_kernel<8>),
+            reinterpret_cast<const void *>(dsplit::decode_split_kernel<16>),
+        };
+        for (const void *k : split_kernels) {
+            if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, optin) != cudaSuccess ||
+                cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+                st.status = W3_ERR_CUDA;
+                return;
+            }
+        }
         const void *sk_kernels[] = {
             reinterpret_cast<const void *>(decode_sk::decode_sk_kernel<1>),
             reinterpret_cast<const void *>(decode_sk::decode_sk_kernel<2>),
@@ -418,12 +433,119 @@ w3_status launch_decode(const uint16_t *x, const int32_t *packed, const uint16_t
     return e == cudaSuccess ? W3_OK : W3_ERR_CUDA;
 }
 
+const void *split_kernel(int mt) {
+    switch (mt) {
+        case 1: return reinterpret_cast<const void *>(dsplit::decode_split_kernel<1>);
+        case 2: return reinterpret_cast<const void *>(dsplit::decode_split_kernel<2>);
+        case 4: return reinterpret_cast<const void *>(dsplit::decode_split_kernel<4>);
+        case 8: return reinterpret_cast<const void *>(dsplit::decode_split_kernel<8>);
+        default: return reinterpret_cast<const void *>(dsplit::decode_split_kernel<16>);
+    }
+}
+
+// Clusters of C CTAs of the split decode (batch padded to mt) with `smem` bytes each that
+// the current device keeps resident at once (0 if the query fails).  Cached per device.
+int split_active_clusters(int mt, int C, int smem) {
+    struct Key {
+        int dev, mt, C, smem, n;
+    };
+    static std::mutex mu;
+    static Key cache[256];
+    static int ncache = 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    {
+        std::lock_guard<std::mutex> g(mu);
+        for (int i = 0; i < ncache; ++i)
+            if (cache[i].dev == dev && cache[i].mt == mt && cache[i].C == C && cache[i].smem == smem) return cache[i].n;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(C, 1, 1);
+    cfg.blockDim = dim3(dsplit::kWarps * 32, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, split_kernel(mt), &cfg) != cudaSuccess) {
+        (void)cudaGetLastError();
+        n = 0;
+    }
+    std::lock_guard<std::mutex> g(mu);
+    if (ncache < 256) cache[ncache++] = {dev, mt, C, smem, n};
+    return n;
+}
+
+dsplit::LaunchPlan split_plan(int M, int N, int K, int sms) {
+    const int mt = decode::padded_batch(M);
+    return dsplit::plan(M, N, K, sms, [&](int C, int smem) { return split_active_clusters(mt, C, smem); });
+}
+
+// The split decode (decode_split.cuh), M <= 16, N >= 32.
+w3_status launch_decode_split(const uint16_t *x, const int32_t *packed, const uint16_t *scales, uint16_t *y, int M,
+                              int N, int K, const dsplit::LaunchPlan &P, cudaStream_t stream) {
+    dsplit::Params prm;
+    const int64_t words = static_cast<int64_t>(K) * 3 / 32;
+    if (w3_status s = encode_packed_map(&prm.tmap1, packed, N, words, dsplit::kPitch1, dsplit::kBlockRows)) return s;
+    const int pitch_s = dsplit::stage_groups_for(P.mt) * kWordsPerGroup;
+    prm.tmapS = prm.tmap1;
+    prm.hasS = words >= pitch_s;
+    if (prm.hasS) {
+        if (w3_status s = encode_packed_map(&prm.tmapS, packed, N, words, pitch_s, dsplit::kBlockRows)) return s;
+    }
+    prm.x = x;
+    prm.scales = scales;
+    prm.y = y;
+    prm.M = M;
+    prm.N = N;
+    prm.K = K;
+    prm.G = K / kGroup;
+    prm.C = P.C;
+    prm.ncl = P.ncl;
+    prm.depth = P.depth;
+    prm.gs_max = P.gs_max;
+    prm.nb_max = P.nb_max;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(P.ncl * P.C, 1, 1);
+    cfg.blockDim = dim3(P.warps() * 32, 1, 1);
+    cfg.dynamicSmemBytes = P.smem_bytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    set_pdl(attr[0]);  // overlaps the set-up with the previous kernel's tail
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (P.C > 1) {
+        attr[1].id = cudaLaunchAttributeClusterDimension;
+        attr[1].val.clusterDim.x = P.C;
+        attr[1].val.clusterDim.y = 1;
+        attr[1].val.clusterDim.z = 1;
+        cfg.numAttrs = 2;
+    }
+    cudaError_t e;
+    switch (P.mt) {
+        case 1: e = cudaLaunchKernelEx(&cfg, dsplit::decode_split_kernel<1>, prm); break;
+        case 2: e = cudaLaunchKernelEx(&cfg, dsplit::decode_split_kernel<2>, prm); break;
+        case 4: e = cudaLaunchKernelEx(&cfg, dsplit::decode_split_kernel<4>, prm); break;
+        case 8: e = cudaLaunchKernelEx(&cfg, dsplit::decode_split_kernel<8>, prm); break;
+        default: e = cudaLaunchKernelEx(&cfg, dsplit::decode_split_kernel<16>, prm); break;
+    }
+    return e == cudaSuccess ? W3_OK : W3_ERR_CUDA;
+}
+
 // ---- kernel selection (host logic only: depends on the shape and the SM count) --------
 
 // Smallest batch that runs on the tensor-core decode (below it the mma.sync decodes).
 constexpr int kTcMinBatch = 5;
+#ifndef W3_SPLIT_MAX_M
+#define W3_SPLIT_MAX_M 16
+#endif
 
 enum class Route {
+    DecodeSplit,    // decode_split_kernel: M <= 16, N >= 32 (cluster split-K, mma.sync)
     DecodeStreamK,  // decode_sk_kernel: M <= 4, at least one 32-row block per SM
     Decode,         // decode_kernel: the remaining small shapes (M <= 16)
     DecodeTc,       // decode_tc_kernel (+ fix-up): 5 <= M <= 16, N >= 256
@@ -435,6 +557,7 @@ enum class Route {
 
 // The route of one pass of at most 16 batch rows.
 Route decode_route(int64_t mb, int64_t N, int64_t K, int sms) {
+    if (N >= dsplit::kBlockRows && mb >= kTcMinBatch && mb <= W3_SPLIT_MAX_M) return Route::DecodeSplit;
     if (N >= decode_tc::kRows && mb >= kTcMinBatch) return Route::DecodeTc;
     if (N >= static_cast<int64_t>(decode_sk::kBlockRows) * sms &&
         decode_sk::applicable(static_cast<int>(mb), static_cast<int>(N), static_cast<int>(K)))
@@ -453,6 +576,7 @@ Route choose_route(int64_t M, int64_t N, int64_t K, int sms) {
 
 const char *route_name(Route r) {
     switch (r) {
+        case Route::DecodeSplit: return "decode_split";
         case Route::DecodeStreamK: return "decode_sk";
         case Route::Decode: return "decode";
         case Route::DecodeTc: return "decode_tc";
@@ -551,6 +675,12 @@ w3_status run_gemm(const uint16_t *x, const int32_t *packed, const uint16_t *sca
         const uint16_t *xp = x + m0 * K;
         uint16_t *yp = y + m0 * N;
         switch (decode_route(mb, N, K, sms)) {
+            case Route::DecodeSplit: {
+                const dsplit::LaunchPlan sp = split_plan(mb, n, k, sms);
+                status = sp.ok ? launch_decode_split(xp, packed, scales, yp, mb, n, k, sp, st)
+                               : launch_decode(xp, packed, scales, yp, mb, n, k, sms, st);
+                break;
+            }
             case Route::DecodeTc:
                 status = launch_decode_tc<decode_tc::Instance>(xp, packed, scales, yp, mb, n, k, tplan, partial, st);
                 break;
