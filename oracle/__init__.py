@@ -75,6 +75,12 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         lib.oracle_gemm_f64_entries.restype = ctypes.c_int
         lib.oracle_weight_row_norms.argtypes = [p, p, i64, i64, p]
         lib.oracle_weight_row_norms.restype = ctypes.c_int
+        lib.oracle_native_words.argtypes = [i64, i64]
+        lib.oracle_native_words.restype = i64
+        for name in ("oracle_native_from_packed", "oracle_packed_from_native"):
+            f = getattr(lib, name)
+            f.argtypes = [p, p, i64, i64]
+            f.restype = ctypes.c_int
         lib.oracle_ct4_words_per_row.argtypes = [i64]
         lib.oracle_ct4_words_per_row.restype = i64
         lib.oracle_pack_ct4.argtypes = [p, p, i64, i64]
@@ -130,6 +136,29 @@ class Oracle:
             raise ValueError("packed width does not match K")
         out = np.empty((N, K), dtype=np.uint8)
         _check(self.lib.oracle_unpack(_ptr(packed), _ptr(out), N, K), "oracle_unpack")
+        return out
+
+    def native_words(self, N: int, K: int) -> int:
+        """Words of the kernel-native block layout of an N x K weight (rows padded to 32)."""
+        return int(self.lib.oracle_native_words(N, K))
+
+    def native_from_packed(self, packed: np.ndarray, K: int) -> np.ndarray:
+        """packed uint32 [N, 3K/32] (row order) -> the native block order, uint32 [native_words]."""
+        packed = _c(packed.view(np.uint32), np.uint32)
+        N = packed.shape[0]
+        if packed.shape[1] != self.words_per_row(K):
+            raise ValueError("packed width does not match K")
+        out = np.empty(max(self.native_words(N, K), 0), dtype=np.uint32)
+        _check(self.lib.oracle_native_from_packed(_ptr(packed), _ptr(out), N, K), "oracle_native_from_packed")
+        return out
+
+    def packed_from_native(self, native: np.ndarray, N: int, K: int) -> np.ndarray:
+        """The inverse: native block order -> packed uint32 [N, 3K/32]."""
+        native = _c(native.view(np.uint32), np.uint32)
+        if native.size != self.native_words(N, K):
+            raise ValueError("native size does not match N, K")
+        out = np.empty((N, max(self.words_per_row(K), 0)), dtype=np.uint32)
+        _check(self.lib.oracle_packed_from_native(_ptr(native), _ptr(out), N, K), "oracle_packed_from_native")
         return out
 
     def ct4_words_per_row(self, K: int) -> int:

@@ -320,3 +320,58 @@ int oracle_repack_ct4(const uint32_t *ct4, uint32_t *packed, int64_t N, int64_t 
     }
     return 0;
 }
+
+/* ---- the kernel-native block layout (a permutation of the packed words) ------------------
+ *
+ * The storage above keeps each row's words together.  The decode kernels read 32 rows at a
+ * time, each of 32 lanes taking one 32-code block (3 words) of each of four rows, so this
+ * library also defines an optional "native" order of the same words (the GLQ page's
+ * decoder-native "kernel" layout is the precedent: an offline re-order of the checkpoint for
+ * the kernel, behind the same format).  Rows are grouped in blocks of 32 (the last block
+ * padded with zero rows); for block b, group g (128 codes), lane l = 4r + c (r = l / 4 in
+ * 0..7, c = l % 4 in 0..3), word 3h + i (h in 0..3, i in 0..2):
+ *     native[((b*G + g)*32 + l)*12 + 3h + i] = packed[row 32b + r + 8h][word 12g + 3c + i]
+ * i.e. lane l holds 32-code block c of group g for rows r, r+8, r+16, r+24, in the row's own
+ * bit order.  Size: ceil(N/32)*32 rows of 3K/32 words.
+ */
+
+/* Words of the native layout for an N x K weight (rows padded to a multiple of 32). */
+int64_t oracle_native_words(int64_t N, int64_t K) {
+    int64_t W = oracle_words_per_row(K);
+    if (N < 0 || W < 0 || K % ORACLE_GROUP != 0) return -1;
+    return (N + 31) / 32 * 32 * W;
+}
+
+/* packed [N, 3K/32] (row order) -> native (block order above); padded rows are zero. */
+int oracle_native_from_packed(const uint32_t *packed, uint32_t *native, int64_t N, int64_t K) {
+    int64_t W = oracle_words_per_row(K), G = oracle_groups_per_row(K), NW = oracle_native_words(N, K);
+    if (!packed || !native || N < 0 || W < 0 || G < 0 || NW < 0) return -1;
+    int64_t NB = (N + 31) / 32;
+    for (int64_t b = 0; b < NB; ++b)
+        for (int64_t g = 0; g < G; ++g)
+            for (int l = 0; l < 32; ++l)
+                for (int h = 0; h < 4; ++h)
+                    for (int i = 0; i < 3; ++i) {
+                        int64_t row = 32 * b + l / 4 + 8 * h;
+                        int64_t word = 12 * g + 3 * (l % 4) + i;
+                        native[((b * G + g) * 32 + l) * 12 + 3 * h + i] = row < N ? packed[row * W + word] : 0u;
+                    }
+    return 0;
+}
+
+/* native -> packed [N, 3K/32] (the inverse; padded rows are dropped). */
+int oracle_packed_from_native(const uint32_t *native, uint32_t *packed, int64_t N, int64_t K) {
+    int64_t W = oracle_words_per_row(K), G = oracle_groups_per_row(K), NW = oracle_native_words(N, K);
+    if (!packed || !native || N < 0 || W < 0 || G < 0 || NW < 0) return -1;
+    int64_t NB = (N + 31) / 32;
+    for (int64_t b = 0; b < NB; ++b)
+        for (int64_t g = 0; g < G; ++g)
+            for (int l = 0; l < 32; ++l)
+                for (int h = 0; h < 4; ++h)
+                    for (int i = 0; i < 3; ++i) {
+                        int64_t row = 32 * b + l / 4 + 8 * h;
+                        int64_t word = 12 * g + 3 * (l % 4) + i;
+                        if (row < N) packed[row * W + word] = native[((b * G + g) * 32 + l) * 12 + 3 * h + i];
+                    }
+    return 0;
+}

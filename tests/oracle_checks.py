@@ -276,6 +276,54 @@ def check_ct4_repack_equals_direct_pack(orc):
     assert np.array_equal(packed, orc.pack(codes))
 
 
+# --- the kernel-native block layout ---------------------------------------------------
+
+def check_native_layout_golden_words(orc):
+    """Hand-derived positions of the native block order (tests/golden/native_layout_words.json)."""
+    g = json.load(open(os.path.join(GOLDEN, "native_layout_words.json")))
+    N, K = g["N"], g["K"]
+    W = orc.words_per_row(K)
+    packed = (1000 * np.arange(N, dtype=np.uint32)[:, None] + np.arange(W, dtype=np.uint32)[None, :] + 1)
+    native = orc.native_from_packed(packed.astype(np.uint32), K)
+    assert native.size == g["native_words"] == orc.native_words(N, K)
+    for e in g["entries"]:
+        assert int(native[e["index"]]) == e["value"], e
+
+
+def check_native_layout_round_trip_and_padding(orc):
+    rng = np.random.Generator(np.random.PCG64(21))
+    for N, K in [(32, 128), (33, 256), (100, 384), (7, 1152)]:
+        packed = orc.pack(rng.integers(0, 8, size=(N, K), dtype=np.uint8))
+        native = orc.native_from_packed(packed, K)
+        assert native.size == -(-N // 32) * 32 * orc.words_per_row(K)
+        assert np.array_equal(orc.packed_from_native(native, N, K), packed)
+        # every word of a real row appears once; padded rows are zero
+        assert np.array_equal(np.sort(native[native != 0]), np.sort(packed[packed != 0].ravel()))
+    assert orc.native_words(5, 100) == -1
+
+
+def check_native_lane_blocks_decode_to_their_rows(orc):
+    """Read as a little-endian 96-bit integer, lane l's words 3h..3h+2 of group g of block b are
+    sum_j c[32b + l/4 + 8h, 128g + 32(l%4) + j] * 8^j (the base-8 form of the row bit order)."""
+    rng = np.random.Generator(np.random.PCG64(22))
+    N, K = 70, 256
+    codes = rng.integers(0, 8, size=(N, K), dtype=np.uint8)
+    native = orc.native_from_packed(orc.pack(codes), K)
+    G = K // 128
+    for b in range(-(-N // 32)):
+        for gg in range(G):
+            for lane in range(32):
+                for h in range(4):
+                    base = ((b * G + gg) * 32 + lane) * 12 + 3 * h
+                    v = int(native[base]) | int(native[base + 1]) << 32 | int(native[base + 2]) << 64
+                    row = 32 * b + lane // 4 + 8 * h
+                    want = 0
+                    if row < N:
+                        for j in range(32):
+                            want += int(codes[row, 128 * gg + 32 * (lane % 4) + j]) * 8 ** j
+                    assert v == want, (b, gg, lane, h)
+
+
 ALL_CHECKS = [
     check_worked_example_shapes,
     check_bits_per_weight,
@@ -292,4 +340,7 @@ ALL_CHECKS = [
     check_rejects_bad_arguments,
     check_ct4_container_words,
     check_ct4_repack_equals_direct_pack,
+    check_native_layout_golden_words,
+    check_native_layout_round_trip_and_padding,
+    check_native_lane_blocks_decode_to_their_rows,
 ]

@@ -33,6 +33,12 @@ MUTANTS = [
      "field |= stream_bit(in, 4 * k + i) << (3 - i);", 1),
     ("ct4_clamp_not_counted", "                q = 3;\n                ++*out_of_range;", "                q = 3;", 1),
     ("ct4_pack_offset_7", "unsigned field = (unsigned)(q + 8);", "unsigned field = (unsigned)(q + 7);", 1),
+    # the native block order, changed the same way in both directions (so the round trip still holds)
+    ("native_lane_row_and_block_swapped", "int64_t row = 32 * b + l / 4 + 8 * h;",
+     "int64_t row = 32 * b + l % 4 + 8 * h;", 2),
+    ("native_row_stride_4", "int64_t row = 32 * b + l / 4 + 8 * h;", "int64_t row = 32 * b + l / 4 + 4 * h;", 2),
+    ("native_words_of_lane_block", "int64_t word = 12 * g + 3 * (l % 4) + i;",
+     "int64_t word = 12 * g + 3 * (l / 8) + i;", 2),
 ]
 
 
