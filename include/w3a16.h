@@ -157,6 +157,51 @@ w3_status w3a16_gemm_noalloc(const uint16_t *x, const int32_t *packed, const uin
                              int64_t M, int64_t N, int64_t K, w3_stream_t stream);
 
 /*
+ * The kernel-native block order (optional).  The decode kernels read a weight
+ * 32 rows at a time, each of 32 lanes taking one 32-code block (3 words) of
+ * four rows.  These calls store the same words permuted so that the words one
+ * decode warp needs for a run of groups are one contiguous range (a single
+ * 1-D bulk copy) and each lane's 12 words of a group are adjacent (three
+ * 16-byte loads).  The GLQ page's decoder-native "kernel" layout
+ * (trellis_layout "kernel") is the precedent: an offline re-order of a
+ * checkpoint for its kernel; the exact-width storage above stays the
+ * interchange format and the bit order inside each 3-word block is unchanged.
+ * Definition: rows are grouped in blocks of 32 (the last padded with zero
+ * rows); for block b, group g (128 codes), lane l = 4r + c (r = l/4 in 0..7,
+ * c = l%4 in 0..3) and word 3h + i (h in 0..3, i in 0..2)
+ *     native[((b*G + g)*32 + l)*12 + 3h + i] = packed[32b + r + 8h][12g + 3c + i],
+ * G = K/128.  Scales keep their [N, K/128] layout.
+ */
+
+/* Words of the native order for an N x K weight: ceil(N/32)*32 * 3K/32; -1 for an invalid shape. */
+int64_t w3_native_words(int64_t N, int64_t K);
+
+/*
+ * w3_pack_native -- codes [N,K] uint8 (0..7) -> native int32 [w3_native_words(N,K)]
+ * (the same words w3_pack writes, in the native order; padded rows zero).
+ * Errors as w3_pack.
+ */
+w3_status w3_pack_native(const uint8_t *codes, int32_t *native, int64_t N, int64_t K, w3_stream_t stream);
+
+/* w3_native_from_packed -- packed [N, 3K/32] -> native order (a permutation of words). Errors as w3_pack. */
+w3_status w3_native_from_packed(const int32_t *packed, int32_t *native, int64_t N, int64_t K, w3_stream_t stream);
+
+/* w3_packed_from_native -- the inverse: native order -> packed [N, 3K/32]. Errors as w3_pack. */
+w3_status w3_packed_from_native(const int32_t *native, int32_t *packed, int64_t N, int64_t K, w3_stream_t stream);
+
+/*
+ * w3a16_gemm_native -- y = x * W^T like w3a16_gemm, with W given in the native
+ * order (scales [N, K/128] as usual), for decode batches: 1 <= M <= 16 and
+ * N >= 32 (W3_ERR_UNSUPPORTED otherwise; larger batches use w3a16_gemm on the
+ * row-major words).  Same arithmetic and determinism as w3a16_gemm's decode
+ * (the weight enters exactly; fp32 accumulation; one rounding to bf16).
+ * Allocates nothing.  Errors: W3_ERR_NULL, W3_ERR_SHAPE, W3_ERR_ALIGN,
+ * W3_ERR_ALIAS, W3_ERR_UNSUPPORTED, W3_ERR_CUDA.
+ */
+w3_status w3a16_gemm_native(const uint16_t *x, const int32_t *native, const uint16_t *scales, uint16_t *y,
+                            int64_t M, int64_t N, int64_t K, w3_stream_t stream);
+
+/*
  * w3a16_gemm_route -- which kernels w3a16_gemm (and w3a16_gemm_noalloc) run for
  * an M x N x K product on a GPU with `num_sms` SMs, as a short name:
  *   "decode_sk"   persistent stream-K mma.sync decode (M <= 4, many rows);

@@ -71,6 +71,22 @@ def test_host_argument_checks(lib):
     assert r(FAKE_A, FAKE_A + 16, 4, 128, NULL, NULL) == 7  # output overlaps the container
 
 
+def test_native_order_host_checks(lib):
+    assert lib.w3_native_words(40, 256) == 64 * 24  # two 32-row blocks of 24 words per row
+    assert lib.w3_native_words(32, 8192) == 32 * 768
+    assert lib.w3_native_words(1, 100) == -1
+    assert lib.w3_pack_native(NULL, FAKE_B, 4, 128, NULL) == 1
+    assert lib.w3_native_from_packed(FAKE_A, FAKE_B, 4, 96, NULL) == 2
+    assert lib.w3_packed_from_native(FAKE_A + 4, FAKE_B, 4, 128, NULL) == 3
+    assert lib.w3_native_from_packed(FAKE_A, FAKE_A + 16, 40, 256, NULL) == 7  # overlap
+    g = lib.w3a16_gemm_native
+    assert g(NULL, FAKE_B, FAKE_C, FAKE_D, 1, 64, 128, NULL) == 1
+    assert g(FAKE_A, FAKE_B, FAKE_C, FAKE_D, 0, 64, 128, NULL) == 2
+    assert g(FAKE_A, FAKE_B, FAKE_C, FAKE_D, 17, 64, 128, NULL) == 5  # batches above 16: row-major path
+    assert g(FAKE_A, FAKE_B, FAKE_C, FAKE_D, 1, 16, 128, NULL) == 5   # fewer than 32 rows
+    assert g(FAKE_A, FAKE_B, FAKE_C, FAKE_B, 1, 64, 128, NULL) == 7   # y overlaps the weights
+
+
 def test_no_silent_fallback_without_a_device(lib):
     import torch
 

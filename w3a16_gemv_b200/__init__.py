@@ -15,11 +15,16 @@ from ._binding import (  # noqa: F401
     w3_check_device_error,
     w3_dequant_f32,
     w3_groups_per_row,
+    w3_native_from_packed,
+    w3_native_words,
     w3_pack,
+    w3_pack_native,
+    w3_packed_from_native,
     w3_packed_words_per_row,
     w3_repack_ct4,
     w3_unpack,
     w3a16_gemm,
+    w3a16_gemm_native,
     w3a16_gemm_noalloc,
     w3a16_gemm_route,
 )
@@ -31,11 +36,16 @@ __all__ = [
     "w3_check_device_error",
     "w3_dequant_f32",
     "w3_groups_per_row",
+    "w3_native_from_packed",
+    "w3_native_words",
     "w3_pack",
+    "w3_pack_native",
+    "w3_packed_from_native",
     "w3_packed_words_per_row",
     "w3_repack_ct4",
     "w3_unpack",
     "w3a16_gemm",
+    "w3a16_gemm_native",
     "w3a16_gemm_noalloc",
     "w3a16_gemm_route",
 ]

@@ -43,6 +43,11 @@ SIGNATURES = [
     ("w3_repack_ct4", ctypes.c_int, [_P, _P, _I64, _I64, _P, _P]),
     ("w3a16_gemm", ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P]),
     ("w3a16_gemm_noalloc", ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P]),
+    ("w3_native_words", _I64, [_I64, _I64]),
+    ("w3_pack_native", ctypes.c_int, [_P, _P, _I64, _I64, _P]),
+    ("w3_native_from_packed", ctypes.c_int, [_P, _P, _I64, _I64, _P]),
+    ("w3_packed_from_native", ctypes.c_int, [_P, _P, _I64, _I64, _P]),
+    ("w3a16_gemm_native", ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P]),
     ("w3a16_gemm_route", ctypes.c_char_p, [_I64, _I64, _I64, ctypes.c_int32]),
     ("w3_check_device_error", ctypes.c_int, [_P]),
 ]
@@ -199,6 +204,75 @@ def _gemm(entry: str, x: torch.Tensor, packed: torch.Tensor, scales: torch.Tenso
         raise ValueError("out must be [M, N]")
     _check(getattr(lib(), entry)(x.data_ptr(), packed.data_ptr(), scales.data_ptr(), out.data_ptr(), M, N, K,
                                  _stream(stream)), entry)
+    return out
+
+
+def w3_native_words(N: int, K: int) -> int:
+    return int(lib().w3_native_words(N, K))
+
+
+def _native_out(N: int, K: int, device, out: torch.Tensor | None) -> torch.Tensor:
+    n = w3_native_words(N, K)
+    if n < 0:
+        raise ValueError(f"no native order for N={N}, K={K}")
+    if out is None:
+        out = torch.empty((n,), dtype=torch.int32, device=device)
+    _need(out, torch.int32, "native")
+    if out.numel() != n:
+        raise ValueError(f"native must hold {n} words")
+    return out
+
+
+def w3_pack_native(codes: torch.Tensor, native: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """codes uint8 [N,K] (0..7) -> the native block order, int32 [w3_native_words(N, K)]."""
+    _need(codes, torch.uint8, "codes")
+    N, K = codes.shape
+    native = _native_out(N, K, codes.device, native)
+    _check(lib().w3_pack_native(codes.data_ptr(), native.data_ptr(), N, K, _stream(stream)), "w3_pack_native")
+    return native
+
+
+def w3_native_from_packed(packed: torch.Tensor, K: int, native: torch.Tensor | None = None, stream=None):
+    """packed int32 [N, 3K/32] -> the native block order (a permutation of the words)."""
+    _need(packed, torch.int32, "packed")
+    N = packed.shape[0]
+    if packed.shape[1] != w3_packed_words_per_row(K):
+        raise ValueError("packed width does not match K")
+    native = _native_out(N, K, packed.device, native)
+    _check(lib().w3_native_from_packed(packed.data_ptr(), native.data_ptr(), N, K, _stream(stream)),
+           "w3_native_from_packed")
+    return native
+
+
+def w3_packed_from_native(native: torch.Tensor, N: int, K: int, packed: torch.Tensor | None = None, stream=None):
+    """The native block order -> packed int32 [N, 3K/32]."""
+    _need(native, torch.int32, "native")
+    if native.numel() != w3_native_words(N, K):
+        raise ValueError("native size does not match N, K")
+    if packed is None:
+        packed = torch.empty((N, w3_packed_words_per_row(K)), dtype=torch.int32, device=native.device)
+    _need(packed, torch.int32, "packed")
+    _check(lib().w3_packed_from_native(native.data_ptr(), packed.data_ptr(), N, K, _stream(stream)),
+           "w3_packed_from_native")
+    return packed
+
+
+def w3a16_gemm_native(x: torch.Tensor, native: torch.Tensor, scales: torch.Tensor, N: int,
+                      out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """y = x W^T with W in the native block order (decode batches, M <= 16)."""
+    _need(x, torch.bfloat16, "x")
+    _need(native, torch.int32, "native")
+    _need(scales, torch.bfloat16, "scales")
+    M, K = x.shape
+    if native.numel() != w3_native_words(N, K) or tuple(scales.shape) != (N, w3_groups_per_row(K)):
+        raise ValueError("native/scales sizes do not match N, K")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _need(out, torch.bfloat16, "out")
+    if tuple(out.shape) != (M, N):
+        raise ValueError("out must be [M, N]")
+    _check(lib().w3a16_gemm_native(x.data_ptr(), native.data_ptr(), scales.data_ptr(), out.data_ptr(), M, N, K,
+                                   _stream(stream)), "w3a16_gemm_native")
     return out
 
 

@@ -71,11 +71,16 @@ w3_status device_setup(int *num_sms, cudaMemPool_t *pool = nullptr) {
             reinterpret_cast<const void *>(decode::decode_kernel<16>),
         };
         const void *split_kernels[] = {
-            reinterpret_cast<const void *>(dsplit::decode_split_kernel<1>),
-            reinterpret_cast<const void *>(dsplit::decode_split_kernel<2>),
-            reinterpret_cast<const void *>(dsplit::decode_split_kernel<4>),
-            reinterpret_cast<const void *>(dsplit::decode_split_kernel<8>),
-            reinterpret_cast<const void *>(dsplit::decode_split_kernel<16>),
+            reinterpret_cast<const void *>(dsplit::decode_split_kernel<1, false>),
+            reinterpret_cast<const void *>(dsplit::decode_split_kernel<2, false>),
+            reinterpret_cast<const void *>(dsplit::decode_split_kernel<4, false>),
+            reinterpret_cast<const void *>(dsplit::decode_split_kernel<8, false>),
+            reinterpret_cast<const void *>(dsplit::decode_split_kernel<16, false>),
+            reinterpret_cast<const void *>(dsplit::decode_split_kernel<1, true>),
+            reinterpret_cast<const void *>(dsplit::decode_split_kernel<2, true>),
+            reinterpret_cast<const void *>(dsplit::decode_split_kernel<4, true>),
+            reinterpret_cast<const void *>(dsplit::decode_split_kernel<8, true>),
+            reinterpret_cast<const void *>(dsplit::decode_split_kernel<16, true>),
         };
         for (const void *k : split_kernels) {
             if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, optin) != cudaSuccess ||
@@ -85,9 +90,12 @@ w3_status device_setup(int *num_sms, cudaMemPool_t *pool = nullptr) {
             }
         }
         const void *sk_kernels[] = {
-            reinterpret_cast<const void *>(decode_sk::decode_sk_kernel<1>),
-            reinterpret_cast<const void *>(decode_sk::decode_sk_kernel<2>),
-            reinterpret_cast<const void *>(decode_sk::decode_sk_kernel<4>),
+            reinterpret_cast<const void *>(decode_sk::decode_sk_kernel<1, false>),
+            reinterpret_cast<const void *>(decode_sk::decode_sk_kernel<2, false>),
+            reinterpret_cast<const void *>(decode_sk::decode_sk_kernel<4, false>),
+            reinterpret_cast<const void *>(decode_sk::decode_sk_kernel<1, true>),
+            reinterpret_cast<const void *>(decode_sk::decode_sk_kernel<2, true>),
+            reinterpret_cast<const void *>(decode_sk::decode_sk_kernel<4, true>),
         };
         for (const void *k : sk_kernels) {
             if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, optin) != cudaSuccess) {
@@ -189,17 +197,23 @@ w3_status encode_packed_map(CUtensorMap *map, const int32_t *packed, int64_t N, 
                : W3_ERR_CUDA;
 }
 
+// The stream-K decode on the row-major words (`packed`) or, when `native` is given, on the
+// same words in the native block order.
 w3_status launch_decode_sk(const uint16_t *x, const int32_t *packed, const uint16_t *scales, uint16_t *y, int M,
-                           int N, int K, int num_sms, cudaStream_t stream) {
+                           int N, int K, int num_sms, cudaStream_t stream, const int32_t *native = nullptr) {
     const decode_sk::LaunchPlan P = decode_sk::plan(M, N, K, num_sms);
     decode_sk::Params prm;
     const int64_t words = static_cast<int64_t>(K) * 3 / 32;
-    if (w3_status s = encode_packed_map(&prm.tmap1, packed, N, words, decode_sk::kPitch1, decode_sk::kBlockRows))
-        return s;
-    prm.tmap3 = prm.tmap1;  // only used when a segment has 3 groups left, which needs K >= 384
-    if (words >= decode_sk::kPitch3) {
-        if (w3_status s = encode_packed_map(&prm.tmap3, packed, N, words, decode_sk::kPitch3, decode_sk::kBlockRows))
+    prm.native = reinterpret_cast<const uint32_t *>(native);
+    if (!native) {
+        if (w3_status s = encode_packed_map(&prm.tmap1, packed, N, words, decode_sk::kPitch1, decode_sk::kBlockRows))
             return s;
+        prm.tmap3 = prm.tmap1;  // only used when a segment has 3 groups left, which needs K >= 384
+        if (words >= decode_sk::kPitch3) {
+            if (w3_status s =
+                    encode_packed_map(&prm.tmap3, packed, N, words, decode_sk::kPitch3, decode_sk::kBlockRows))
+                return s;
+        }
     }
     prm.x = x;
     prm.scales = scales;
@@ -219,10 +233,18 @@ w3_status launch_decode_sk(const uint16_t *x, const int32_t *packed, const uint1
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     cudaError_t e;
-    switch (P.mt) {
-        case 1: e = cudaLaunchKernelEx(&cfg, decode_sk::decode_sk_kernel<1>, prm); break;
-        case 2: e = cudaLaunchKernelEx(&cfg, decode_sk::decode_sk_kernel<2>, prm); break;
-        default: e = cudaLaunchKernelEx(&cfg, decode_sk::decode_sk_kernel<4>, prm); break;
+    if (native) {
+        switch (P.mt) {
+            case 1: e = cudaLaunchKernelEx(&cfg, decode_sk::decode_sk_kernel<1, true>, prm); break;
+            case 2: e = cudaLaunchKernelEx(&cfg, decode_sk::decode_sk_kernel<2, true>, prm); break;
+            default: e = cudaLaunchKernelEx(&cfg, decode_sk::decode_sk_kernel<4, true>, prm); break;
+        }
+    } else {
+        switch (P.mt) {
+            case 1: e = cudaLaunchKernelEx(&cfg, decode_sk::decode_sk_kernel<1, false>, prm); break;
+            case 2: e = cudaLaunchKernelEx(&cfg, decode_sk::decode_sk_kernel<2, false>, prm); break;
+            default: e = cudaLaunchKernelEx(&cfg, decode_sk::decode_sk_kernel<4, false>, prm); break;
+        }
     }
     return e == cudaSuccess ? W3_OK : W3_ERR_CUDA;
 }
@@ -435,11 +457,11 @@ w3_status launch_decode(const uint16_t *x, const int32_t *packed, const uint16_t
 
 const void *split_kernel(int mt) {
     switch (mt) {
-        case 1: return reinterpret_cast<const void *>(dsplit::decode_split_kernel<1>);
-        case 2: return reinterpret_cast<const void *>(dsplit::decode_split_kernel<2>);
-        case 4: return reinterpret_cast<const void *>(dsplit::decode_split_kernel<4>);
-        case 8: return reinterpret_cast<const void *>(dsplit::decode_split_kernel<8>);
-        default: return reinterpret_cast<const void *>(dsplit::decode_split_kernel<16>);
+        case 1: return reinterpret_cast<const void *>(dsplit::decode_split_kernel<1, false>);
+        case 2: return reinterpret_cast<const void *>(dsplit::decode_split_kernel<2, false>);
+        case 4: return reinterpret_cast<const void *>(dsplit::decode_split_kernel<4, false>);
+        case 8: return reinterpret_cast<const void *>(dsplit::decode_split_kernel<8, false>);
+        default: return reinterpret_cast<const void *>(dsplit::decode_split_kernel<16, false>);
     }
 }
 
@@ -485,17 +507,23 @@ dsplit::LaunchPlan split_plan(int M, int N, int K, int sms) {
     return dsplit::plan(M, N, K, sms, [&](int C, int smem) { return split_active_clusters(mt, C, smem); });
 }
 
-// The split decode (decode_split.cuh), M <= 16, N >= 32.
+// The split decode (decode_split.cuh), M <= 16, N >= 32, on the row-major words (`packed`)
+// or, when `native` is given, on the native block order.
 w3_status launch_decode_split(const uint16_t *x, const int32_t *packed, const uint16_t *scales, uint16_t *y, int M,
-                              int N, int K, const dsplit::LaunchPlan &P, cudaStream_t stream) {
+                              int N, int K, const dsplit::LaunchPlan &P, cudaStream_t stream,
+                              const int32_t *native = nullptr) {
     dsplit::Params prm;
     const int64_t words = static_cast<int64_t>(K) * 3 / 32;
-    if (w3_status s = encode_packed_map(&prm.tmap1, packed, N, words, dsplit::kPitch1, dsplit::kBlockRows)) return s;
+    prm.native = reinterpret_cast<const uint32_t *>(native);
     const int pitch_s = dsplit::stage_groups_for(P.mt) * kWordsPerGroup;
-    prm.tmapS = prm.tmap1;
     prm.hasS = words >= pitch_s;
-    if (prm.hasS) {
-        if (w3_status s = encode_packed_map(&prm.tmapS, packed, N, words, pitch_s, dsplit::kBlockRows)) return s;
+    if (!native) {
+        if (w3_status s = encode_packed_map(&prm.tmap1, packed, N, words, dsplit::kPitch1, dsplit::kBlockRows))
+            return s;
+        prm.tmapS = prm.tmap1;
+        if (prm.hasS) {
+            if (w3_status s = encode_packed_map(&prm.tmapS, packed, N, words, pitch_s, dsplit::kBlockRows)) return s;
+        }
     }
     prm.x = x;
     prm.scales = scales;
@@ -526,12 +554,22 @@ w3_status launch_decode_split(const uint16_t *x, const int32_t *packed, const ui
         cfg.numAttrs = 2;
     }
     cudaError_t e;
-    switch (P.mt) {
-        case 1: e = cudaLaunchKernelEx(&cfg, dsplit::decode_split_kernel<1>, prm); break;
-        case 2: e = cudaLaunchKernelEx(&cfg, dsplit::decode_split_kernel<2>, prm); break;
-        case 4: e = cudaLaunchKernelEx(&cfg, dsplit::decode_split_kernel<4>, prm); break;
-        case 8: e = cudaLaunchKernelEx(&cfg, dsplit::decode_split_kernel<8>, prm); break;
-        default: e = cudaLaunchKernelEx(&cfg, dsplit::decode_split_kernel<16>, prm); break;
+    if (native) {
+        switch (P.mt) {
+            case 1: e = cudaLaunchKernelEx(&cfg, dsplit::decode_split_kernel<1, true>, prm); break;
+            case 2: e = cudaLaunchKernelEx(&cfg, dsplit::decode_split_kernel<2, true>, prm); break;
+            case 4: e = cudaLaunchKernelEx(&cfg, dsplit::decode_split_kernel<4, true>, prm); break;
+            case 8: e = cudaLaunchKernelEx(&cfg, dsplit::decode_split_kernel<8, true>, prm); break;
+            default: e = cudaLaunchKernelEx(&cfg, dsplit::decode_split_kernel<16, true>, prm); break;
+        }
+    } else {
+        switch (P.mt) {
+            case 1: e = cudaLaunchKernelEx(&cfg, dsplit::decode_split_kernel<1, false>, prm); break;
+            case 2: e = cudaLaunchKernelEx(&cfg, dsplit::decode_split_kernel<2, false>, prm); break;
+            case 4: e = cudaLaunchKernelEx(&cfg, dsplit::decode_split_kernel<4, false>, prm); break;
+            case 8: e = cudaLaunchKernelEx(&cfg, dsplit::decode_split_kernel<8, false>, prm); break;
+            default: e = cudaLaunchKernelEx(&cfg, dsplit::decode_split_kernel<16, false>, prm); break;
+        }
     }
     return e == cudaSuccess ? W3_OK : W3_ERR_CUDA;
 }
@@ -706,6 +744,19 @@ w3_status check_gemm_args(const uint16_t *x, const int32_t *packed, const uint16
     return W3_OK;
 }
 
+// y = x W^T on the native block order (validated arguments): M <= 16, N >= 32.
+w3_status run_gemm_native(const uint16_t *x, const int32_t *native, const uint16_t *scales, uint16_t *y,
+                          int64_t M, int64_t N, int64_t K, int sms, cudaStream_t st) {
+    const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
+    if (M <= 4 && N >= static_cast<int64_t>(decode_sk::kBlockRows) * sms && decode_sk::applicable(m, n, k))
+        return launch_decode_sk(x, nullptr, scales, y, m, n, k, sms, st, native);
+    const dsplit::LaunchPlan sp = split_plan(m, n, k, sms);
+    if (!sp.ok) return W3_ERR_UNSUPPORTED;
+    return launch_decode_split(x, nullptr, scales, y, m, n, k, sp, st, native);
+}
+
+int64_t native_words(int64_t N, int64_t K) { return (N + 31) / 32 * 32 * (K * 3 / 32); }
+
 #ifdef W3_TEST_HOOKS
 // Test-only: one thread waits, with the bounded wait every kernel uses, on an
 // mbarrier phase that nothing completes, so the wait runs out and records the
@@ -832,6 +883,62 @@ w3_status w3a16_gemm_noalloc(const uint16_t *x, const int32_t *packed, const uin
     scratch.fixed_floats = kNoAllocScratchFloats;
     if (!scratch.fixed) return W3_ERR_CUDA;
     return run_gemm(x, packed, scales, y, M, N, K, sms, reinterpret_cast<cudaStream_t>(stream), scratch);
+}
+
+int64_t w3_native_words(int64_t N, int64_t K) { return check_nk(N, K) == W3_OK ? native_words(N, K) : -1; }
+
+// The three conversions of the native block order: one thread per 3-word block.
+static w3_status native_convert(int kind, const void *src, void *dst, int64_t N, int64_t K, w3_stream_t stream) {
+    if (!src || !dst) return W3_ERR_NULL;
+    if (w3_status s = check_nk(N, K)) return s;
+    if (!aligned16(src) || !aligned16(dst)) return W3_ERR_ALIGN;
+    const int64_t nwords = native_words(N, K), rwords = N * K * 3 / 32;
+    const int64_t src_bytes = kind == 0 ? N * K : kind == 1 ? rwords * 4 : nwords * 4;
+    const int64_t dst_bytes = kind == 2 ? rwords * 4 : nwords * 4;
+    if (overlaps(src, src_bytes, dst, dst_bytes)) return W3_ERR_ALIAS;
+    int sms;
+    if (w3_status s = device_setup(&sms)) return s;
+    const int64_t nthreads = nwords / 3;
+    const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (kind == 0)
+        pack_native_kernel<<<grid_for(nthreads, 256), 256, 0, st>>>(static_cast<const uint8_t *>(src),
+                                                                    static_cast<uint32_t *>(dst), N, K, nthreads);
+    else if (kind == 1)
+        native_from_packed_kernel<<<grid_for(nthreads, 256), 256, 0, st>>>(static_cast<const uint32_t *>(src),
+                                                                           static_cast<uint32_t *>(dst), N, K,
+                                                                           nthreads);
+    else
+        packed_from_native_kernel<<<grid_for(nthreads, 256), 256, 0, st>>>(static_cast<const uint32_t *>(src),
+                                                                           static_cast<uint32_t *>(dst), N, K,
+                                                                           nthreads);
+    return launch_status();
+}
+
+w3_status w3_pack_native(const uint8_t *codes, int32_t *native, int64_t N, int64_t K, w3_stream_t stream) {
+    return native_convert(0, codes, native, N, K, stream);
+}
+
+w3_status w3_native_from_packed(const int32_t *packed, int32_t *native, int64_t N, int64_t K, w3_stream_t stream) {
+    return native_convert(1, packed, native, N, K, stream);
+}
+
+w3_status w3_packed_from_native(const int32_t *native, int32_t *packed, int64_t N, int64_t K, w3_stream_t stream) {
+    return native_convert(2, native, packed, N, K, stream);
+}
+
+w3_status w3a16_gemm_native(const uint16_t *x, const int32_t *native, const uint16_t *scales, uint16_t *y, int64_t M,
+                            int64_t N, int64_t K, w3_stream_t stream) {
+    if (!x || !native || !scales || !y) return W3_ERR_NULL;
+    if (w3_status s = check_nk(N, K)) return s;
+    if (M < 1 || M > 16 || N < 32) return M < 1 ? W3_ERR_SHAPE : W3_ERR_UNSUPPORTED;
+    if (!aligned16(x) || !aligned16(native) || !aligned16(scales) || !aligned16(y)) return W3_ERR_ALIGN;
+    const int64_t ybytes = M * N * 2;
+    if (overlaps(y, ybytes, x, M * K * 2) || overlaps(y, ybytes, native, native_words(N, K) * 4) ||
+        overlaps(y, ybytes, scales, N * (K / kGroup) * 2))
+        return W3_ERR_ALIAS;
+    int sms;
+    if (w3_status s = device_setup(&sms)) return s;
+    return run_gemm_native(x, native, scales, y, M, N, K, sms, reinterpret_cast<cudaStream_t>(stream));
 }
 
 const char *w3a16_gemm_route(int64_t M, int64_t N, int64_t K, int32_t num_sms) {

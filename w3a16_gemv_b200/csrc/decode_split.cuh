@@ -20,8 +20,11 @@
 // deterministic, and no global scratch or atomic is used.
 //
 // Loads: each warp streams its range through a private ring of tiled TMA
-// copies, [32 rows x 36 words] (3 groups) or [32 rows x 12 words] boxes.
-// Batches of 9..16 rows use two n8 MMA tiles per k-step.
+// copies, [32 rows x 36 words] (3 groups) or [32 rows x 12 words] boxes; with
+// the kernel-native block order (NATIVE; see format_kernels.cuh) a stage is one
+// 1-D bulk copy of a block's consecutive groups and a lane reads its 12 words
+// of a group with three 16-byte shared-memory loads.  Batches of 9..16 rows use
+// two n8 MMA tiles per k-step.
 #pragma once
 
 #include "decode_gemv.cuh"
@@ -39,7 +42,8 @@ constexpr int kBlockRows = 32;  // rows per warp block (two 16-row MMA tiles)
 constexpr int kMaxStageGroups = 3;
 constexpr int kPitch1 = kWordsPerGroup;                       // 12 words: rows of a 1-group box
 __host__ __device__ constexpr int stage_bytes(int mt) { return kBlockRows * stage_groups_for(mt) * kWordsPerGroup * 4; }
-constexpr int kBox1Bytes = kBlockRows * kPitch1 * 4;          // 1536
+constexpr int kBox1Bytes = kBlockRows * kPitch1 * 4;          // 1536: one group of a block
+constexpr int kNativeGroupWords = kBlockRows * kPitch1;       // 384
 constexpr int kSmemLimit = 227 * 1024;
 constexpr int kMaxCluster = 8;
 static_assert(kBlockRows * 2 * kWordsPerGroup * 4 % 128 == 0 && kBlockRows * 3 * kWordsPerGroup * 4 % 128 == 0 &&
@@ -71,6 +75,7 @@ __host__ __device__ inline SmemLayout smem_layout(int gs, int mt, int depth, int
 struct Params {
     CUtensorMap tmapS;  // packed [N][3K/32] u32, box [32 rows][12 * stage groups words]
     CUtensorMap tmap1;  // same tensor, box [32 rows][12 words]
+    const uint32_t *native;  // the same words in the native block order (NATIVE kernels)
     const uint16_t *x;
     const uint16_t *scales;
     uint16_t *y;
@@ -121,7 +126,7 @@ __device__ __forceinline__ void ksteps(const uint32_t (&w)[JN][4][3], const uint
 // JN consecutive groups (1 or 3) of one 32-row block: group j of the stage is
 // row i, word k at st[i*pitch + j*jstride_w + k]; xs_g points at the first
 // group's prepared x; the group's scales multiply the fp32 results into acc.
-template <int JN, int MT, int NT>
+template <int JN, int MT, int NT, bool NATIVE>
 __device__ __forceinline__ void groups(const uint32_t *st, int pitch, int jstride_w, int grel, int gabs,
                                        const uint2 *xs_lane, const float4 *ncorr, const uint16_t *const (&sc)[4],
                                        int r, int c, float (&acc)[2][NT][4], uint32_t magic) {
@@ -132,11 +137,21 @@ __device__ __forceinline__ void groups(const uint32_t *st, int pitch, int jstrid
         for (int h = 0; h < 4; ++h) s[j][h] = bf16_bits_to_f32(__ldg(sc[h] + gabs + j));
     uint32_t w[JN][4][3];  // block c of group j in rows r, r+8, r+16, r+24
 #pragma unroll
-    for (int j = 0; j < JN; ++j)
+    for (int j = 0; j < JN; ++j) {
+        if constexpr (NATIVE) {
+            const uint4 *q = reinterpret_cast<const uint4 *>(st + j * kNativeGroupWords + (4 * r + c) * 12);
+            const uint4 a = q[0], b = q[1], e = q[2];
+            w[j][0][0] = a.x; w[j][0][1] = a.y; w[j][0][2] = a.z;
+            w[j][1][0] = a.w; w[j][1][1] = b.x; w[j][1][2] = b.y;
+            w[j][2][0] = b.z; w[j][2][1] = b.w; w[j][2][2] = e.x;
+            w[j][3][0] = e.y; w[j][3][1] = e.z; w[j][3][2] = e.w;
+        } else {
 #pragma unroll
-        for (int h = 0; h < 4; ++h)
+            for (int h = 0; h < 4; ++h)
 #pragma unroll
-            for (int i = 0; i < 3; ++i) w[j][h][i] = st[(8 * h + r) * pitch + j * jstride_w + 3 * c + i];
+                for (int i = 0; i < 3; ++i) w[j][h][i] = st[(8 * h + r) * pitch + j * jstride_w + 3 * c + i];
+        }
+    }
     float d[JN][2][NT][4];
 #pragma unroll
     for (int j = 0; j < JN; ++j)
@@ -177,7 +192,7 @@ __device__ __forceinline__ void store_frag(uint16_t *y, int N, int M, int block,
     }
 }
 
-template <int MT>
+template <int MT, bool NATIVE>
 __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(const __grid_constant__ Params p) {
     static_assert(MT == 1 || MT == 2 || MT == 4 || MT == 8 || MT == 16, "batch rows padded to 1, 2, 4, 8, 16");
     constexpr int NT = n_tiles(MT);
@@ -244,7 +259,13 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(const __gr
         if (lane == 0) {
             const uint32_t bar = bar0 + 8 * slot;
             const uint32_t dst = ring0 + slot * kStageBytes;
-            if (ng == kStageGroups && p.hasS) {
+            if constexpr (NATIVE) {
+                // ng consecutive groups of one block: one contiguous range
+                mbar_arrive_expect_tx(bar, ng * kBox1Bytes);
+                bulk_copy_g2s(dst,
+                              p.native + (static_cast<int64_t>(row0 / kBlockRows) * G + gq0 + g) * kNativeGroupWords,
+                              ng * kBox1Bytes, bar);
+            } else if (ng == kStageGroups && p.hasS) {
                 mbar_arrive_expect_tx(bar, kStageBytes);
                 tma_load_2d(dst, &p.tmapS, (gq0 + g) * kWordsPerGroup, row0, bar);
             } else {
@@ -350,13 +371,13 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(const __gr
         ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar0 + 8 * slot, parity) && ok);
         if (ok) {
             const uint32_t *st = reinterpret_cast<const uint32_t *>(ring + slot * kStageBytes);
-            if (ng == kStageGroups && p.hasS) {
-                groups<kStageGroups, MT, NT>(st, kPitchS, kWordsPerGroup, cg, gq0 + cg, xs_lane, ncorr, sc, r, c, acc,
-                                             magic);
+            if (ng == kStageGroups && (NATIVE || p.hasS)) {
+                groups<kStageGroups, MT, NT, NATIVE>(st, kPitchS, kWordsPerGroup, cg, gq0 + cg, xs_lane, ncorr, sc, r,
+                                                     c, acc, magic);
             } else {
                 for (int j = 0; j < ng; ++j)
-                    groups<1, MT, NT>(st + j * kBlockRows * kPitch1, kPitch1, 0, cg + j, gq0 + cg + j, xs_lane, ncorr,
-                                      sc, r, c, acc, magic);
+                    groups<1, MT, NT, NATIVE>(st + j * kBlockRows * kPitch1, kPitch1, 0, cg + j, gq0 + cg + j, xs_lane,
+                                              ncorr, sc, r, c, acc, magic);
             }
         }
         // End of a segment.  A whole block is emitted.  A split block is either this warp's

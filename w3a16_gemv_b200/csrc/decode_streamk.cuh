@@ -18,6 +18,10 @@
 // the 32 rows, fetched with one tiled TMA copy ([32 rows][36 words] box, dense,
 // conflict-free pitch); a stage with 1 or 2 groups left in its segment uses
 // 1-group boxes ([32][12 words]) so that no byte outside the range is read.
+// With the kernel-native block order (NATIVE; see format_kernels.cuh) a stage
+// of a block's consecutive groups is one contiguous range of memory, fetched
+// with a single 1-D bulk copy, and each lane reads its 12 words of a group with
+// three 16-byte shared-memory loads (lane-ordered, free of bank conflicts).
 #pragma once
 
 #include "decode_gemv.cuh"
@@ -27,21 +31,16 @@ namespace decode_sk {
 
 using decode::unpack_block;
 
-#ifndef W3_SK_WARPS
-#define W3_SK_WARPS 12
-#endif
-#ifndef W3_SK_MAX_DEPTH
-#define W3_SK_MAX_DEPTH 4
-#endif
-constexpr int kWarps = W3_SK_WARPS;
-constexpr int kMaxDepth = W3_SK_MAX_DEPTH;  // ring stages per warp; the launch picks 2..kMaxDepth
+constexpr int kWarps = 12;
+constexpr int kMaxDepth = 4;  // ring stages per warp; the launch picks 2..kMaxDepth
 constexpr int kTileRows = 16;
 constexpr int kBlockRows = 32;                           // rows per warp block (2 tiles)
 constexpr int kStageGroups = 3;
 constexpr int kPitch3 = kStageGroups * kWordsPerGroup;   // 36 words: rows of a 3-group box
 constexpr int kPitch1 = kWordsPerGroup;                  // 12 words: rows of a 1-group box
 constexpr int kStageBytes = kBlockRows * kPitch3 * 4;    // 4608
-constexpr int kBox1Bytes = kBlockRows * kPitch1 * 4;     // 1536
+constexpr int kBox1Bytes = kBlockRows * kPitch1 * 4;     // 1536: one group of a block (also in the native order)
+constexpr int kNativeGroupWords = kBlockRows * kPitch1;  // 384
 constexpr int kXsBudgetBytes = 96 * 1024;
 constexpr int kSmemLimit = 227 * 1024;
 static_assert(kStageBytes % 128 == 0 && kBox1Bytes % 128 == 0,
@@ -67,6 +66,7 @@ __host__ __device__ inline SmemLayout smem_layout(int G, int mt, int depth) {
 struct Params {
     CUtensorMap tmap3;  // packed [N][3K/32] u32, box [32 rows][36 words]
     CUtensorMap tmap1;  // same tensor, box [32 rows][12 words]
+    const uint32_t *native;  // the same words in the native block order (NATIVE kernels)
     const uint16_t *x;
     const uint16_t *scales;
     uint16_t *y;
@@ -104,19 +104,36 @@ __device__ __forceinline__ void block_ksteps(const uint32_t (&w)[4][3], const ui
     }
 }
 
+// The 12 words of lane (r, c) for group j of a stage (block c of the group in rows
+// r, r+8, r+16, r+24): row i, word w of group j at st[i*pitch + j*jstride + w] in
+// a row-major box, or lane-ordered in the native order.
+template <bool NATIVE>
+__device__ __forceinline__ void lane_words(const uint32_t *st, int pitch, int jstride, int j, int r, int c,
+                                           uint32_t (&w)[4][3]) {
+    if constexpr (NATIVE) {
+        const uint4 *q = reinterpret_cast<const uint4 *>(st + j * kNativeGroupWords + (4 * r + c) * 12);
+        const uint4 a = q[0], b = q[1], d = q[2];
+        w[0][0] = a.x; w[0][1] = a.y; w[0][2] = a.z;
+        w[1][0] = a.w; w[1][1] = b.x; w[1][2] = b.y;
+        w[2][0] = b.z; w[2][1] = b.w; w[2][2] = d.x;
+        w[3][0] = d.y; w[3][1] = d.z; w[3][2] = d.w;
+    } else {
+#pragma unroll
+        for (int h = 0; h < 4; ++h)
+#pragma unroll
+            for (int i = 0; i < 3; ++i) w[h][i] = st[(8 * h + r) * pitch + j * jstride + 3 * c + i];
+    }
+}
+
 // One group of one 32-row block: both tiles' 8 MMAs as two interleaved chains,
-// each started from the group's -corr and scaled in fp32 into acc.  Row i,
-// word w of group j of the stage is st[i*pitch + j*jstride + w].
-template <int MT>
+// each started from the group's -corr and scaled in fp32 into acc.
+template <int MT, bool NATIVE>
 __device__ __forceinline__ void block_group(const uint32_t *st, int pitch, int jstride, int j, int gabs,
                                             const uint2 *xs_lane, const float4 *ncorr,
                                             const uint16_t *const (&sc)[4], int r, int c,
                                             float (&acc)[2][4], uint32_t magic) {
     uint32_t w[4][3];  // block c of the group in rows r, r+8, r+16, r+24
-#pragma unroll
-    for (int h = 0; h < 4; ++h)
-#pragma unroll
-        for (int i = 0; i < 3; ++i) w[h][i] = st[(8 * h + r) * pitch + j * jstride + 3 * c + i];
+    lane_words<NATIVE>(st, pitch, jstride, j, r, c, w);
     const float4 nc = ncorr[gabs * 4];
     float d0[4] = {nc.x, nc.y, nc.z, nc.w};
     float d1[4] = {nc.x, nc.y, nc.z, nc.w};
@@ -155,7 +172,7 @@ __device__ __forceinline__ void stage_ksteps(const uint32_t (&w)[3][4][3], const
     }
 }
 
-template <int MT>
+template <int MT, bool NATIVE>
 __device__ __forceinline__ void full_stage(const uint32_t *st, int g, const uint2 *xs_lane, const float4 *ncorr,
                                            const uint16_t *const (&sc)[4], int r, int c,
                                            float (&acc)[2][4], uint32_t magic) {
@@ -166,11 +183,7 @@ __device__ __forceinline__ void full_stage(const uint32_t *st, int g, const uint
         for (int h = 0; h < 4; ++h) s[j][h] = bf16_bits_to_f32(__ldg(sc[h] + g + j));
     uint32_t w[3][4][3];
 #pragma unroll
-    for (int j = 0; j < 3; ++j)
-#pragma unroll
-        for (int h = 0; h < 4; ++h)
-#pragma unroll
-            for (int i = 0; i < 3; ++i) w[j][h][i] = st[(8 * h + r) * kPitch3 + j * kWordsPerGroup + 3 * c + i];
+    for (int j = 0; j < 3; ++j) lane_words<NATIVE>(st, kPitch3, kWordsPerGroup, j, r, c, w[j]);
     float d[3][2][4];
 #pragma unroll
     for (int j = 0; j < 3; ++j) {
@@ -207,7 +220,7 @@ __device__ __forceinline__ void store_block(uint16_t *y, int N, int M, int block
         }
 }
 
-template <int MT>
+template <int MT, bool NATIVE>
 __global__ void __launch_bounds__(kWarps * 32, 1) decode_sk_kernel(const __grid_constant__ Params p) {
     static_assert(MT == 1 || MT == 2 || MT == 4, "stream-K decode handles batches up to 4");
     extern __shared__ __align__(128) uint8_t smem[];
@@ -271,7 +284,12 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_sk_kernel(const __grid_
         if (lane == 0) {
             const uint32_t bar = bar0 + 8 * slot;
             const uint32_t dst = ring0 + slot * kStageBytes;
-            if (ng == kStageGroups) {
+            if constexpr (NATIVE) {
+                // ng consecutive groups of one block: one contiguous range
+                mbar_arrive_expect_tx(bar, ng * kBox1Bytes);
+                bulk_copy_g2s(dst, p.native + (static_cast<int64_t>(row0 / kBlockRows) * G + g) * kNativeGroupWords,
+                              ng * kBox1Bytes, bar);
+            } else if (ng == kStageGroups) {
                 mbar_arrive_expect_tx(bar, kStageBytes);
                 tma_load_2d(dst, &p.tmap3, g * kWordsPerGroup, row0, bar);
             } else {
@@ -367,11 +385,11 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_sk_kernel(const __grid_
         if (ok) {
             const uint32_t *st = reinterpret_cast<const uint32_t *>(ring + slot * kStageBytes);
             if (ng == kStageGroups) {
-                full_stage<MT>(st, cg, xs_lane, ncorr, sc, r, c, acc, magic);
+                full_stage<MT, NATIVE>(st, cg, xs_lane, ncorr, sc, r, c, acc, magic);
             } else {
                 for (int j = 0; j < ng; ++j)
-                    block_group<MT>(st, kPitch1, kBlockRows * kPitch1, j, cg + j, xs_lane, ncorr, sc, r, c, acc,
-                                    magic);
+                    block_group<MT, NATIVE>(st, kPitch1, kBlockRows * kPitch1, j, cg + j, xs_lane, ncorr, sc, r, c,
+                                            acc, magic);
             }
         }
         // end of a segment: store a whole block, or park a partial one in a slot

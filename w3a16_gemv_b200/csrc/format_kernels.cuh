@@ -115,3 +115,82 @@ __global__ void __launch_bounds__(256) repack_ct4_kernel(const uint4 *__restrict
 }
 
 }  // namespace w3
+
+namespace w3 {
+
+// The kernel-native block order of the packed words (the decode kernels read 32 rows
+// at a time, each lane one 32-code block of four rows): rows in blocks of 32 (the
+// last padded with zero rows); for block b, group g, lane l = 4r + c, word 3h + i:
+//     native[((b*G + g)*32 + l)*12 + 3h + i] = packed[row 32b + r + 8h][word 12g + 3c + i].
+// One thread moves one 3-word block (t -> h = t % 4, l = t/4 % 32, g, b), so the
+// writes of a warp are contiguous.
+__device__ __forceinline__ void native_coords(int64_t t, int64_t G, int64_t &row, int64_t &word) {
+    const int h = static_cast<int>(t & 3), l = static_cast<int>((t >> 2) & 31);
+    const int64_t bg = t >> 7, g = bg % G, b = bg / G;
+    row = 32 * b + (l >> 2) + 8 * h;
+    word = 12 * g + 3 * (l & 3);
+}
+
+__global__ void __launch_bounds__(256) native_from_packed_kernel(const uint32_t *__restrict__ packed,
+                                                                 uint32_t *__restrict__ native, int64_t N,
+                                                                 int64_t K, int64_t nthreads) {
+    const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (t >= nthreads) return;
+    const int64_t W = K * 3 / 32, G = K / kGroup;
+    int64_t row, word;
+    native_coords(t, G, row, word);
+    uint32_t v[3] = {0u, 0u, 0u};
+    if (row < N) {
+        const uint32_t *src = packed + row * W + word;
+        v[0] = src[0];
+        v[1] = src[1];
+        v[2] = src[2];
+    }
+    uint32_t *dst = native + 3 * t;
+    dst[0] = v[0];
+    dst[1] = v[1];
+    dst[2] = v[2];
+}
+
+__global__ void __launch_bounds__(256) packed_from_native_kernel(const uint32_t *__restrict__ native,
+                                                                 uint32_t *__restrict__ packed, int64_t N,
+                                                                 int64_t K, int64_t nthreads) {
+    const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (t >= nthreads) return;
+    const int64_t W = K * 3 / 32, G = K / kGroup;
+    int64_t row, word;
+    native_coords(t, G, row, word);
+    if (row >= N) return;
+    const uint32_t *src = native + 3 * t;
+    uint32_t *dst = packed + row * W + word;
+    dst[0] = src[0];
+    dst[1] = src[1];
+    dst[2] = src[2];
+}
+
+// codes [N,K] -> native directly: the 3 words of (row, 32-code block) packed as in
+// pack_kernel and written at their native position.
+__global__ void __launch_bounds__(256) pack_native_kernel(const uint8_t *__restrict__ codes,
+                                                          uint32_t *__restrict__ native, int64_t N, int64_t K,
+                                                          int64_t nthreads) {
+    const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (t >= nthreads) return;
+    const int64_t G = K / kGroup;
+    int64_t row, word;
+    native_coords(t, G, row, word);
+    unsigned __int128 v = 0;
+    if (row < N) {
+        // word 12g + 3c is 32-code block 4g + c of the row: codes 32 * (word / 3) ...
+        const uint4 *src = reinterpret_cast<const uint4 *>(codes + row * K + 32 * (word / 3));
+        uint4 q[2] = {src[0], src[1]};
+        const uint8_t *c = reinterpret_cast<const uint8_t *>(q);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v |= static_cast<unsigned __int128>(c[j] & 7u) << (3 * j);
+    }
+    uint32_t *dst = native + 3 * t;
+    dst[0] = static_cast<uint32_t>(v);
+    dst[1] = static_cast<uint32_t>(v >> 32);
+    dst[2] = static_cast<uint32_t>(v >> 64);
+}
+
+}  // namespace w3
