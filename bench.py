@@ -60,7 +60,6 @@ ROUTE_KERNELS = {
     "decode_split": "w3::dsplit::decode_split_kernel",
     "decode_sk": "w3::decode_sk::decode_sk_kernel",
     "decode": "w3::decode::decode_kernel",
-    "decode_tc": "w3::decode_tc::decode_tc_kernel",
     "decode_tc32": "w3::decode_tc32::decode_tc_kernel",
     "prefill": "w3::prefill::prefill_kernel",
     "prefill_ab": "w3::prefill_ab::prefill_ab_kernel",
@@ -81,9 +80,10 @@ def kernel_name(M: int, N: int, K: int, sms: int) -> str:
 
 
 def kernels_per_call(M: int, N: int, K: int, sms: int) -> int:
-    """Kernels one w3a16_gemm call launches: the tensor-core decode routes are followed by their
-    partial-sum fix-up kernel when the work is split over more than one CTA (always, at these sizes)."""
-    return 2 if route(M, N, K, sms) in ("decode_tc", "decode_tc32") else 1
+    """Kernels one w3a16_gemm call launches: the 32-wide tensor-core decode is followed by its
+    partial-sum fix-up kernel when the work is split over more than one CTA (always, at these
+    sizes); every other route is one kernel."""
+    return 2 if route(M, N, K, sms) == "decode_tc32" else 1
 
 
 def step_bytes() -> int:

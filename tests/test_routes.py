@@ -11,7 +11,7 @@ from w3a16_gemv_b200 import _binding, build, w3a16_gemm_route
 
 SMS = 148  # B200
 
-ROUTES = {"decode_split", "decode_sk", "decode", "decode_tc", "decode_tc32", "prefill", "prefill_ab", "passes"}
+ROUTES = {"decode_split", "decode_sk", "decode", "decode_tc32", "prefill", "prefill_ab", "passes"}
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -41,7 +41,7 @@ def test_every_shape_has_a_known_route(M, N, K):
         assert r in ("decode_sk", "decode")
     if r == "decode_sk":
         assert M <= 4 and N >= 32 * SMS
-    if r in ("decode_tc", "decode_tc32"):
+    if r == "decode_tc32":
         assert N >= 256
     if r == "decode_tc32":
         assert 17 <= M <= 32

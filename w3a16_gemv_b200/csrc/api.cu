@@ -16,10 +16,7 @@
 #include "decode_gemv.cuh"
 #include "decode_split.cuh"
 #include "decode_streamk.cuh"
-// the tensor-core decode, once per batch width (16: M <= 16; 32: 17 <= M <= 32)
-#include "decode_tcgen05.cuh"
-#undef W3_TC_NS
-#undef W3_TC_BATCH
+// the tensor-core decode for 17 <= M <= 32 (32 batch columns)
 #define W3_TC_NS decode_tc32
 #define W3_TC_BATCH 32
 #include "decode_tcgen05.cuh"
@@ -103,7 +100,7 @@ w3_status device_setup(int *num_sms, cudaMemPool_t *pool = nullptr) {
                 return;
             }
         }
-        if (decode_tc::Instance::set_smem() != cudaSuccess || decode_tc32::Instance::set_smem() != cudaSuccess) {
+        if (decode_tc32::Instance::set_smem() != cudaSuccess) {
             st.status = W3_ERR_CUDA;
             return;
         }
@@ -576,17 +573,13 @@ w3_status launch_decode_split(const uint16_t *x, const int32_t *packed, const ui
 
 // ---- kernel selection (host logic only: depends on the shape and the SM count) --------
 
-// Smallest batch that runs on the tensor-core decode (below it the mma.sync decodes).
-constexpr int kTcMinBatch = 5;
-#ifndef W3_SPLIT_MAX_M
-#define W3_SPLIT_MAX_M 16
-#endif
+// Smallest batch of the split decode (below it, on many rows, the stream-K decode).
+constexpr int kSplitMinBatch = 5;
 
 enum class Route {
     DecodeSplit,    // decode_split_kernel: M <= 16, N >= 32 (cluster split-K, mma.sync)
     DecodeStreamK,  // decode_sk_kernel: M <= 4, at least one 32-row block per SM
     Decode,         // decode_kernel: the remaining small shapes (M <= 16)
-    DecodeTc,       // decode_tc_kernel (+ fix-up): 5 <= M <= 16, N >= 256
     DecodeTc32,     // decode_tc32 decode_tc_kernel (+ fix-up): 17 <= M <= 32, N >= 256
     Prefill,        // prefill_kernel: M > 16 (not on the 32-wide decode), K >= 256
     PrefillAb,      // prefill_ab_kernel: chosen over prefill_kernel per shape
@@ -595,8 +588,7 @@ enum class Route {
 
 // The route of one pass of at most 16 batch rows.
 Route decode_route(int64_t mb, int64_t N, int64_t K, int sms) {
-    if (N >= dsplit::kBlockRows && mb >= kTcMinBatch && mb <= W3_SPLIT_MAX_M) return Route::DecodeSplit;
-    if (N >= decode_tc::kRows && mb >= kTcMinBatch) return Route::DecodeTc;
+    if (N >= dsplit::kBlockRows && mb >= kSplitMinBatch) return Route::DecodeSplit;
     if (N >= static_cast<int64_t>(decode_sk::kBlockRows) * sms &&
         decode_sk::applicable(static_cast<int>(mb), static_cast<int>(N), static_cast<int>(K)))
         return Route::DecodeStreamK;
@@ -617,7 +609,6 @@ const char *route_name(Route r) {
         case Route::DecodeSplit: return "decode_split";
         case Route::DecodeStreamK: return "decode_sk";
         case Route::Decode: return "decode";
-        case Route::DecodeTc: return "decode_tc";
         case Route::DecodeTc32: return "decode_tc32";
         case Route::Prefill: return "prefill";
         case Route::PrefillAb: return "prefill_ab";
@@ -630,7 +621,7 @@ const char *route_name(Route r) {
 // decode for up to kNoAllocMaxCtas CTAs (one per SM).  Every slot the fix-up
 // kernel reads is written by the main kernel of the same call, so nothing in
 // it has to start at zero.
-constexpr int kNoAllocMaxCtas = 160 * decode_tc::kCtasPerSm;
+constexpr int kNoAllocMaxCtas = 160 * decode_tc32::kCtasPerSm;
 constexpr int64_t kNoAllocScratchFloats = int64_t(kNoAllocMaxCtas) * 2 * decode_tc32::kBatch * decode_tc32::kRows;
 static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchFloats];
 
@@ -698,15 +689,7 @@ w3_status run_gemm(const uint16_t *x, const int32_t *packed, const uint16_t *sca
         return status;
     }
     // Decode routes, in passes of at most 16 batch rows (one pass unless M > 16 with K < 256,
-    // where no prefill kernel fits); the tensor-core passes share one scratch buffer.
-    const decode_tc::LaunchPlan tplan = decode_tc::plan(N, K, sms);
-    bool any_tc = false;
-    for (int64_t m0 = 0; m0 < M; m0 += 16)
-        any_tc = any_tc || decode_route(std::min<int64_t>(16, M - m0), N, K, sms) == Route::DecodeTc;
-    float *partial = nullptr;
-    if (any_tc) {
-        if (w3_status s = scratch.acquire(tplan.ws_floats, st, &partial)) return s;
-    }
+    // where no prefill kernel fits).
     w3_status status = W3_OK;
     for (int64_t m0 = 0; m0 < M && status == W3_OK; m0 += 16) {
         const int mb = static_cast<int>(std::min<int64_t>(16, M - m0));
@@ -719,14 +702,10 @@ w3_status run_gemm(const uint16_t *x, const int32_t *packed, const uint16_t *sca
                                : launch_decode(xp, packed, scales, yp, mb, n, k, sms, st);
                 break;
             }
-            case Route::DecodeTc:
-                status = launch_decode_tc<decode_tc::Instance>(xp, packed, scales, yp, mb, n, k, tplan, partial, st);
-                break;
             case Route::DecodeStreamK: status = launch_decode_sk(xp, packed, scales, yp, mb, n, k, sms, st); break;
             default: status = launch_decode(xp, packed, scales, yp, mb, n, k, sms, st); break;
         }
     }
-    if (w3_status s = scratch.release(partial, st); s && status == W3_OK) status = s;
     return status;
 }
 

@@ -40,22 +40,10 @@ namespace decode {
 constexpr int kTileRows = 16;                       // rows of one MMA tile
 constexpr int kTilesPerWarp = 2;
 constexpr int kRowsPerWarp = kTileRows * kTilesPerWarp;  // 32: one bulk copy per lane per stage
-#ifndef W3_DECODE_WARPS
-#define W3_DECODE_WARPS 2
-#endif
-#ifndef W3_DECODE_DEPTH
-#define W3_DECODE_DEPTH 4
-#endif
-#ifndef W3_DECODE_STAGE_GROUPS
-#define W3_DECODE_STAGE_GROUPS 3
-#endif
-#ifndef W3_DECODE_MIN_CTAS
-#define W3_DECODE_MIN_CTAS 4
-#endif
-constexpr int kWarps = W3_DECODE_WARPS;             // warps per CTA
+constexpr int kWarps = 2;                           // warps per CTA
 constexpr int kRowsPerCta = kRowsPerWarp * kWarps;  // 64
-constexpr int kStageGroups = W3_DECODE_STAGE_GROUPS;  // groups per stage (odd: conflict-free row pitch)
-constexpr int kDepth = W3_DECODE_DEPTH;             // ring stages per warp
+constexpr int kStageGroups = 3;                     // groups per stage (odd: conflict-free row pitch)
+constexpr int kDepth = 4;                           // ring stages per warp
 static_assert(kStageGroups % 2 == 1, "an odd number of groups per stage keeps the row pitch conflict-free");
 constexpr int kRowPitchWords = kStageGroups * kWordsPerGroup;   // 36 for 3 groups
 constexpr int kStageBytes = kRowsPerWarp * kRowPitchWords * 4;  // 4608 for 3 groups
@@ -248,7 +236,7 @@ __device__ __forceinline__ void prepare_x(const Params &p, uint8_t *smem, const 
 }
 
 template <int MT>
-__global__ void __launch_bounds__(kWarps * 32, W3_DECODE_MIN_CTAS) decode_kernel(const __grid_constant__ Params p) {
+__global__ void __launch_bounds__(kWarps * 32, 4) decode_kernel(const __grid_constant__ Params p) {
     constexpr int NT = (MT + 7) / 8;
     extern __shared__ __align__(128) uint8_t smem[];
     const int M = p.M, N = p.N;

@@ -1,10 +1,10 @@
-// decode_tcgen05.cuh -- y = x * W^T for M <= 16 on the 5th-generation tensor
+// decode_tcgen05.cuh -- y = x * W^T for 17 <= M <= 32 on the 5th-generation tensor
 // cores, W in the exact-width uint3 / group-128 / bf16-scale format of the GSQ
 // model card ("Storage layout" section), never materialised in memory.
 //
 // The roles of the operands are swapped with respect to a GEMM over the batch:
 // the weights are the MMA's M dimension (two 128-row tiles per CTA) and the
-// batch is its N dimension (16 columns; rows of x beyond M read as zeros and
+// batch is its N dimension (W3_TC_BATCH columns; rows of x beyond M read as zeros and
 // their columns of the result are never stored).  The unpack of a weight is
 // done once whatever M is, and the tensor cores do all of the multiply-adds.
 //
@@ -17,7 +17,7 @@
 //  * Loads (one warp): per stage of up to 3 groups, one tiled TMA copy of the
 //    packed words of the CTA's 256 rows ([256 rows][36 words], or one
 //    [256 rows][12 words] copy per group) and two copies of x per group
-//    ([16 rows][64 k], 128-byte swizzle: the UMMA B-operand layout).  The same
+//    ([W3_TC_BATCH rows][64 k], 128-byte swizzle: the UMMA B operand).  The same
 //    warp then permutes each 32-k block of x in place into the order of the
 //    unpack below (byte permutes, no arithmetic).  A second warp copies the
 //    stage's group scales (256 rows x up to 3) into a shared-memory ring, so
@@ -32,20 +32,20 @@
 //    tensor-memory lane (two tcgen05.st): the A operand.
 //  * One warp per tile, on different SM sub-partitions, issues 8 tcgen05.mma
 //    per group from an elected lane (A from tensor memory, B = permuted x from
-//    shared memory) into a fresh per-group fp32 accumulator of 16 columns (four
+//    shared memory) into a fresh per-group fp32 accumulator of W3_TC_BATCH columns (four
 //    buffers per tile).  The issue of these short MMAs shares its sub-partition
 //    with two row warps and is what paces the kernel, hence one warp per tile.
-//  * The row threads read each group's 16 results back two groups later
+//  * The row threads read each group's results back two groups later
 //    (tcgen05.ld) and add s[n,g] * D to fp32 registers: the group scale is
 //    applied in fp32 and nothing is rounded before the bf16 store.
-// The file is compiled once per batch width, in its own namespace: W3_TC_NS
-// names the instance and W3_TC_BATCH is its UMMA N, 16 (M <= 16) or 32
-// (17 <= M <= 32).  Without them it is the 16-wide instance, decode_tc.
+// The file is compiled in its own namespace: W3_TC_NS names the instance and
+// W3_TC_BATCH is its UMMA N (the library builds decode_tc32, 32 columns, for
+// batches of 17..32 rows; up to 16 rows the mma.sync decodes are faster).
 #ifndef W3_TC_NS
-#define W3_TC_NS decode_tc
+#define W3_TC_NS decode_tc32
 #endif
 #ifndef W3_TC_BATCH
-#define W3_TC_BATCH 16
+#define W3_TC_BATCH 32
 #endif
 
 #include "common.cuh"
@@ -70,16 +70,9 @@ constexpr int kRows = kTiles * kTileRows;         // 256 rows per CTA (one TMA b
 constexpr int kBatch = W3_TC_BATCH;               // UMMA N
 static_assert(kBatch == 16 || kBatch == 32, "batch widths 16 and 32");
 constexpr int kStageGroups = 3;
-// Resident CTAs per SM and, with them, the per-CTA budgets of shared and
-// tensor memory: one CTA with 4 stages and 3 A buffers per tile, or two CTAs
-// with 2 stages and 1 A buffer per tile each (twice the row warps per SM).
-#ifndef W3_DECODE_TC_CTAS_PER_SM
-#define W3_DECODE_TC_CTAS_PER_SM 1
-#endif
-constexpr int kCtasPerSm = W3_DECODE_TC_CTAS_PER_SM;
-static_assert(kCtasPerSm == 1 || kCtasPerSm == 2, "one or two CTAs per SM");
-static_assert(kBatch == 16 || kCtasPerSm == 1, "the 32-wide instance needs the one-CTA budget");
-constexpr int kStages = kBatch == 32 ? 3 : kCtasPerSm == 1 ? 4 : 2;
+// One resident CTA per SM: it takes the shared and tensor memory budgets below.
+constexpr int kCtasPerSm = 1;
+constexpr int kStages = kBatch == 32 ? 3 : 4;
 constexpr int kPitch3 = kStageGroups * kWordsPerGroup;        // 36 words: rows of a 3-group box
 constexpr int kPitch1 = kWordsPerGroup;                       // 12 words: rows of a 1-group box
 constexpr int kBox1Bytes = kRows * kPitch1 * 4;               // 12 KB
@@ -87,7 +80,7 @@ constexpr int kXBox = kBatch * 64 * 2;                        // 2 or 4 KB: [bat
 constexpr int kXGroupBytes = 2 * kXBox;                       // 4 KB
 constexpr int kXBytes = kStageGroups * kXGroupBytes;          // 12 KB
 constexpr int kStageBytes = kXBytes + kStageGroups * kBox1Bytes;  // 48 KB
-constexpr int kABuf = kBatch == 32 ? 2 : kCtasPerSm == 1 ? 3 : 1;  // A buffers (one group each) per tile
+constexpr int kABuf = kBatch == 32 ? 2 : 3;                   // A buffers (one group each) per tile
 constexpr int kDBuf = 4;                                      // accumulators per tile
 constexpr int kLag = 2;                                       // groups between MMA and read-back
 constexpr int kACols = 64;                                    // 128 codes, two bf16 per column
@@ -101,10 +94,7 @@ constexpr int kMmaWarp1 = 3 + kRowWarps;                      // warp 11: the MM
 constexpr int kThreads = (4 + kRowWarps) * 32;                // load, MMA x 2, row warps, scale warp
 constexpr int kScaleSlotBytes = kStageGroups * kRows * 2;     // [3 groups][256 rows] bf16
 
-#ifndef W3_DECODE_TC_MIN_UNITS
-#define W3_DECODE_TC_MIN_UNITS 6
-#endif
-constexpr int kMinUnitsPerCta = W3_DECODE_TC_MIN_UNITS;
+constexpr int kMinUnitsPerCta = 6;  // (tile, group) units per CTA at least
 static_assert(kXGroupBytes % 1024 == 0 && kXBytes % 1024 == 0 && kStageBytes % 1024 == 0,
               "swizzled x boxes need 1024-byte alignment");
 static_assert(kBox1Bytes % 128 == 0, "tiled TMA destinations need 128-byte alignment");
