@@ -626,6 +626,56 @@ def fused_layer(calls, copies, steps, stream, total_bytes):
             "cuda_graph_us_per_replay": g_us, "GB/s": total_bytes / (g_us * 1e-6) / 1e9}
 
 
+def measure_native_step(p, steps: int, dev) -> dict:
+    """The headline decode step (gate_proj, M = 1, 4, 16) on the kernel-native block order of the
+    same weights (w3_native_from_packed, done once, outside the timed region): the step back to
+    back, and each call back to back on its own, device time with CUDA events."""
+    import torch
+
+    from w3a16_gemv_b200 import w3_check_device_error, w3_native_from_packed, w3_pack, w3a16_gemm_native
+
+    natives = [w3_native_from_packed(w3_pack(torch.from_numpy(p.codes).to(dev)), K_COLS)]
+    natives += [natives[0].clone() for _ in range(ROTATE - 1)]
+    sc0 = torch.from_numpy(p.scales_bf16.view(np.int16)).view(torch.bfloat16).to(dev)
+    scs = [sc0] + [sc0.clone() for _ in range(ROTATE - 1)]
+    x_all = torch.from_numpy(p.x_bf16.view(np.int16)).view(torch.bfloat16).to(dev)
+    xs = {m: x_all[:m].contiguous() for m in BATCHES}
+    ys = {m: torch.empty((m, N_ROWS), dtype=torch.bfloat16, device=dev) for m in BATCHES}
+    stream = torch.cuda.current_stream()
+    peak, _ = measured_peak()
+
+    def call(i, j, m):
+        c = (i * len(BATCHES) + j) % ROTATE
+        w3a16_gemm_native(xs[m], natives[c], scs[c], N_ROWS, out=ys[m])
+
+    for i in range(ROTATE):
+        for j, m in enumerate(BATCHES):
+            call(i, j, m)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(steps):
+        for j, m in enumerate(BATCHES):
+            call(i, j, m)
+    b.record(stream)
+    torch.cuda.synchronize()
+    step_ms = a.elapsed_time(b) / steps
+    calls = []
+    for j, m in enumerate(BATCHES):
+        a.record(stream)
+        for i in range(steps):
+            call(i, j, m)
+        b.record(stream)
+        torch.cuda.synchronize()
+        us = a.elapsed_time(b) * 1e3 / steps
+        byt = algorithmic_bytes(m, N_ROWS, K_COLS)
+        calls.append({"M": m, "us_mean": us, "GB/s": byt / (us * 1e-6) / 1e9,
+                      "frac_of_peak": byt / (us * 1e-6) / 1e9 / peak})
+    w3_check_device_error()
+    return {"workload": WORKLOAD + ", weights in the kernel-native block order (w3a16_gemm_native)",
+            "GB/s": step_bytes() / (step_ms * 1e-3) / 1e9, "ms_per_step": step_ms, "steps": steps, "calls": calls}
+
+
 def run_gpu(args):
     import torch
 
@@ -688,10 +738,25 @@ def run_gpu(args):
     w3_check_device_error()
     elapsed_ms = t_start.elapsed_time(t_end)
 
-    # ---- per-call breakdown (second timed pass, at least 200 steps): an event pair around every
-    #      call, which also keeps consecutive calls from overlapping; the roofline's per-launch time
-    #      comes from here ----
+    # ---- per-call breakdown, two ways (further timed passes, at least 200 calls each):
+    #      stream: each call of the step launched back to back on its own (rotating weight copies,
+    #        programmatic dependent launch, as in the step), one event pair around the whole run:
+    #        the mean launch duration the roofline uses;
+    #      isolated: an event pair around every call of the step, which also keeps consecutive
+    #        calls from overlapping ----
     brk_steps = max(200, min(args.steps, 500))
+    stream_us = {}
+    for j, m in enumerate(BATCHES):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for i in range(ROTATE):
+            w3a16_gemm(xs[m], packs[i], scales[i], out=ys[m])
+        a.record(stream)
+        for i in range(brk_steps):
+            c = (i * calls_per_step + j) % ROTATE
+            w3a16_gemm(xs[m], packs[c], scales[c], out=ys[m])
+        b.record(stream)
+        torch.cuda.synchronize()
+        stream_us[m] = a.elapsed_time(b) * 1e3 / brk_steps
     events = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
                for _ in BATCHES] for _ in range(brk_steps)]
     for i in range(brk_steps):
@@ -710,14 +775,16 @@ def run_gpu(args):
     peak, peak_src = measured_peak()
     calls = []
     for m in BATCHES:
-        us = 1e3 * statistics.mean(per_call_ms[m])
+        us = stream_us[m]
+        iso = 1e3 * statistics.mean(per_call_ms[m])
         b = algorithmic_bytes(m, N_ROWS, K_COLS)
         q = np.percentile(np.array(per_call_ms[m]) * 1e3, [10, 90])
         calls.append({"M": m, "kernel": kernel_name(m, N_ROWS, K_COLS, sms), "us_mean": us,
-                      "us_median": 1e3 * statistics.median(per_call_ms[m]),
-                      "us_p10": float(q[0]), "us_p90": float(q[1]),
+                      "us_isolated_mean": iso, "us_isolated_median": 1e3 * statistics.median(per_call_ms[m]),
+                      "us_isolated_p10": float(q[0]), "us_isolated_p90": float(q[1]),
                       "GB/s": b / (us * 1e-6) / 1e9, "TFLOP/s": 2.0 * m * N_ROWS * K_COLS / (us * 1e-6) / 1e12,
-                      "frac_of_peak": b / (us * 1e-6) / 1e9 / peak, "share": 0.0})
+                      "frac_of_peak": b / (us * 1e-6) / 1e9 / peak,
+                      "frac_of_peak_isolated": b / (iso * 1e-6) / 1e9 / peak, "share": 0.0})
     tot = sum(c["us_mean"] for c in calls)
     for c in calls:
         c["share"] = c["us_mean"] / tot
@@ -726,7 +793,10 @@ def run_gpu(args):
                 "frac": dom["GB/s"] / peak, "traffic": recorded_traffic(dom["M"]),
                 "kernel": dom["kernel"],
                 "algorithmic_bytes_per_launch": algorithmic_bytes(dom["M"], N_ROWS, K_COLS),
-                "launch_time": f"mean of {brk_steps} CUDA-event pairs around the call, on the launch stream",
+                "launch_time": f"mean over {brk_steps} launches of the call back to back (rotating weight copies, "
+                               "programmatic dependent launch as in the step), CUDA events on the launch stream; "
+                               "frac_isolated: the same call with an event pair around each launch",
+                "frac_isolated": dom["frac_of_peak_isolated"],
                 "peak_source": peak_src}
 
     # ---- end to end through the public API with host buffers ----
@@ -796,6 +866,7 @@ def run_gpu(args):
         time.sleep(0.02)
         configs = {"1_gemv_4096": measure_sweep("gemv4096", 50, 5, dev, cs),
                    "2_gate_decode": {"workload": WORKLOAD, "see": "value, calls, roofline of this line"},
+                   "2n_gate_decode_native": measure_native_step(p, brk_steps, dev),
                    "3_down_proj": measure_sweep("down", 50, 5, dev, cs),
                    "4_layer": measure_sweep("layer", 50, 5, dev, cs),
                    "5_prefill_2048": measure_prefill(2048, 20, 3, dev, 1, cs)}

@@ -141,10 +141,11 @@ w3_status w3a16_gemm(const uint16_t *x, const int32_t *packed, const uint16_t *s
 /*
  * w3a16_gemm_noalloc -- the same product y = x * W^T as w3a16_gemm, with the
  * same arguments, checks, errors and results, that allocates nothing: the
- * tensor-core decode (5 <= M <= 32, N >= 256) keeps its fp32 partial sums in a
- * fixed scratch array inside the library (about 10.5 MB of device memory per
- * device, sized for up to 160 SMs) instead of a stream-ordered allocation;
- * every other shape runs exactly as in w3a16_gemm.  The format paper has no
+ * 32-wide tensor-core decode (route "decode_tc32": 17 <= M <= 32, N >= 256)
+ * keeps its fp32 partial sums in a fixed scratch array inside the library
+ * (about 10.5 MB of device memory per device, sized for up to 160 SMs) instead
+ * of a stream-ordered allocation; every other route allocates nothing in
+ * either call and runs exactly as in w3a16_gemm.  The format paper has no
  * counterpart to this call; it is for callers that may not allocate.
  *   - W3_ERR_UNSUPPORTED if the decode would need more scratch than the array
  *     holds (a GPU with more than 160 SMs).
@@ -204,10 +205,12 @@ w3_status w3a16_gemm_native(const uint16_t *x, const int32_t *native, const uint
 /*
  * w3a16_gemm_route -- which kernels w3a16_gemm (and w3a16_gemm_noalloc) run for
  * an M x N x K product on a GPU with `num_sms` SMs, as a short name:
- *   "decode_sk"   persistent stream-K mma.sync decode (M <= 4, many rows);
+ *   "decode_split" mma.sync decode, K split over a thread-block cluster with a
+ *                 fixed-order reduction in distributed shared memory
+ *                 (5 <= M <= 16, N >= 32);
+ *   "decode_sk"   persistent stream-K mma.sync decode (M <= 4, N >= 32 * num_sms);
  *   "decode"      mma.sync decode with cluster split-K (the other M <= 16 shapes);
- *   "decode_tc"   tensor-core (tcgen05) decode, 16 columns (5 <= M <= 16, N >= 256);
- *   "decode_tc32" the same, 32 columns (17 <= M <= 32, N >= 256);
+ *   "decode_tc32" tensor-core (tcgen05) decode, 32 columns (17 <= M <= 32, N >= 256);
  *   "prefill"     tcgen05 GEMM, weights dequantized into shared memory;
  *   "prefill_ab"  tcgen05 GEMM, weights dequantized into tensor memory;
  *   "passes"      M > 16 with K < 256: the decode routes on 16-row slices of x.

@@ -5,8 +5,9 @@
   of the fp64 oracle.
 Small shapes are checked in full (several tiles, ragged edges, every decode
 batch size).  The full-size decode workloads (every M <= 16 configuration the
-benchmark times) are checked in full against the oracle; the M = 2048 and
-M = 1024 prefill workloads on 64 whole rows of y plus 4096 sampled entries.
+benchmark times, and the mid-batch ones) are checked in full against the oracle;
+the M = 2048, 1024 and 512 prefill workloads on 64 whole rows of y plus 4096
+sampled entries.
 Position probes (x = e_k) go through every kernel route, each asserted with
 w3a16_gemm_route, so that a bit-order or placement mistake in any one kernel
 shows up as a wrong weight in a known place.
@@ -73,9 +74,28 @@ SMALL = [
     (20, 1000, 4224, "gsq_5level", "absnormal", "normal_outliers"),
     (24, 28672, 256, "uniform8", "lognormal", "normal"),          # many row tiles, two groups
     (31, 300, 8192, "uniform8", "lognormal", "normal"),
-    # the shared-memory prefill with a ragged second 128-row batch tile and a ragged last W tile
     (200, 1000, 1024, "gsq_5level", "absnormal", "normal_outliers"),
     (129, 600, 512, "uniform8", "lognormal", "normal"),
+]
+
+# (route, M, N, K, codes, scales, x): shapes the dispatch sends to a given prefill kernel
+# (asserted with w3a16_gemm_route), checked in full.
+ROUTED = [
+    # the shared-memory prefill: one 128-row MMA tile of x; a ragged second one; a ragged third
+    # 256-row batch tile; four batch tiles; ragged last W tiles (N = 20001)
+    ("prefill", 33, 20001, 256, "uniform8", "lognormal", "normal"),
+    ("prefill", 200, 20001, 256, "gsq_5level", "absnormal", "normal_outliers"),
+    ("prefill", 129, 20001, 512, "uniform8", "lognormal", "normal"),
+    ("prefill", 600, 20480, 256, "uniform8", "absnormal", "normal"),
+    ("prefill", 1024, 8192, 256, "gsq_uniform", "lognormal", "normal"),
+    # the tensor-memory prefill below 256 rows of x (UMMA N = M rounded up to 16) and above
+    ("prefill_ab", 33, 1000, 1024, "uniform8", "lognormal", "normal"),
+    ("prefill_ab", 64, 8192, 512, "gsq_5level", "absnormal", "normal_outliers"),
+    ("prefill_ab", 128, 4096, 1024, "uniform8", "lognormal", "normal"),
+    ("prefill_ab", 255, 600, 512, "uniform8", "lognormal", "normal_outliers"),
+    ("prefill_ab", 200, 1000, 1024, "gsq_uniform", "absnormal", "normal"),
+    ("prefill_ab", 300, 1000, 1024, "uniform8", "lognormal", "normal"),
+    ("prefill_ab", 1100, 8192, 256, "uniform8", "lognormal", "normal"),
 ]
 
 
@@ -85,6 +105,16 @@ def _id(c):
 
 @pytest.mark.parametrize("case", SMALL, ids=[_id(c) for c in SMALL])
 def test_small_shapes_full_parity(orc, case):
+    _full_parity(orc, case)
+
+
+@pytest.mark.parametrize("case", ROUTED, ids=[f"{c[0]}_{_id(c[1:])}" for c in ROUTED])
+def test_prefill_routes_full_parity(orc, case):
+    assert w3a16_gemm_route(*case[1:4]) == case[0]
+    _full_parity(orc, case[1:])
+
+
+def _full_parity(orc, case):
     M, N, K, cd, sd, xd = case
     p = make_problem(M, N, K, cd, sd, xd, seed=11)
     x, codes, scales = device_problem(p)
@@ -96,7 +126,7 @@ def test_small_shapes_full_parity(orc, case):
     assert np.array_equal(w.view(np.uint32), orc.dequant_f32(ref_packed, p.scales_bf16, K).view(np.uint32))
     y = w3a16_gemm(x, packed, scales)
     w3_check_device_error()
-    ref = orc.gemm_f64(p.x_bf16, ref_packed, p.scales_bf16)
+    ref = orc.gemm_f64(p.x_bf16, ref_packed, p.scales_bf16, threads=0)
     tol = bound(p.x_bf16, orc.weight_row_norms(ref_packed, p.scales_bf16, K), K)
     assert_within_bound(from_dev_bf16(y), ref, tol, _id(case))
 
@@ -173,7 +203,9 @@ PROBES = [
     ("decode_split", 16, 512, 384),
     ("decode_split", 16, 40, 128),
     ("decode_tc32", 32, 300, 512),
-    ("prefill", 64, 300, 256),
+    ("prefill", 64, 20001, 256),
+    ("prefill", 300, 20480, 256),
+    ("prefill_ab", 33, 1000, 256),
     ("prefill_ab", 256, 1024, 1024),
     ("passes", 40, 300, 128),
 ]
@@ -261,3 +293,9 @@ def test_prefill_tensor_memory_kernel_full_size_rows_and_entries(orc):
     # M = 1024 on gate_proj: the weights-in-tensor-memory prefill kernel is the one launched
     assert w3a16_gemm_route(1024, 28672, 8192) == "prefill_ab"
     _rows_and_entries_check(orc, "prefill_1024x28672x8192")
+
+
+def test_prefill_shared_memory_kernel_full_size_rows_and_entries(orc):
+    # M = 512 on gate_proj: the shared-memory prefill kernel is the one launched
+    assert w3a16_gemm_route(512, 28672, 8192) == "prefill"
+    _rows_and_entries_check(orc, "prefill_512x28672x8192")

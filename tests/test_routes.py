@@ -36,7 +36,9 @@ def test_every_shape_has_a_known_route(M, N, K):
     r = w3a16_gemm_route(M, N, K, num_sms=SMS)
     assert r in ROUTES
     if 5 <= M <= 16:
-        assert r == ("decode_split" if N >= 32 else "decode")
+        # the split decode wherever its shared memory holds a K slice of x, a ring and the
+        # cluster's partial sums; the older cluster decode otherwise
+        assert r in (("decode_split", "decode") if N >= 32 else ("decode",))
     if M <= 4:
         assert r in ("decode_sk", "decode")
     if r == "decode_sk":
@@ -61,6 +63,48 @@ def test_benchmarked_shapes():
     # fewer 32-row blocks than SMs at M <= 4: the mma.sync decode with cluster split-K
     assert w3a16_gemm_route(1, 1024, 8192, SMS) == "decode"
     assert w3a16_gemm_route(8, 20, 8192, SMS) == "decode"
+
+
+def test_split_decode_where_its_plan_fits():
+    for M in (5, 8, 12, 16):
+        for N, K in ((28672, 8192), (8192, 8192), (1024, 8192), (4096, 4096), (300, 1152)):
+            assert w3a16_gemm_route(M, N, K, SMS) == "decode_split", (M, N, K)
+    assert w3a16_gemm_route(8, 8192, 28672, SMS) == "decode_split"
+    # 16 batch rows over K = 28672: x of an eighth of K, the ring and the partial sums do not fit
+    assert w3a16_gemm_route(16, 8192, 28672, SMS) == "decode"
+    # one SM: no cluster split, and x of the whole K range does not fit
+    assert w3a16_gemm_route(16, 4096, 8192, 1) == "decode"
+    assert w3a16_gemm_route(16, 4096, 1024, 1) == "decode_split"
+
+
+# (M, N, K) -> the faster prefill kernel on B200 (each timed alone, device time per call)
+MEASURED_PREFILL = {
+    (64, 8192, 8192): "prefill_ab",      # 42.4 us against 66.5
+    (256, 8192, 28672): "prefill_ab",    # 139.6 against 254.5
+    (256, 4096, 4096): "prefill_ab",     # 27.9 against 42.1
+    (256, 1024, 8192): "prefill_ab",     # 46.1 against 77.2
+    (64, 28672, 8192): "prefill",        # 81.0 against 84.8
+    (128, 28672, 8192): "prefill",       # 82.0 against 90.6
+    (160, 28672, 8192): "prefill_ab",    # 91.7 against 101.9
+    (512, 28672, 8192): "prefill",       # 197.5 against 228.7
+    (1024, 28672, 8192): "prefill_ab",   # 421.7 against 479.8
+    (3072, 28672, 8192): "prefill_ab",   # 1214.3 against 1393.8
+    (1024, 8192, 28672): "prefill",      # 353.5 against 421.9
+    (1024, 8192, 8192): "prefill",       # 109.3 against 118.5
+    (256, 57344, 8192): "prefill",       # 196.7 against 215.9
+}
+
+
+@pytest.mark.parametrize("shape", sorted(MEASURED_PREFILL))
+def test_prefill_dispatch_picks_the_measured_faster_kernel(shape):
+    assert w3a16_gemm_route(*shape, SMS) == MEASURED_PREFILL[shape]
+
+
+@pytest.mark.parametrize("M", [33, 64, 100, 128, 160, 200, 255, 256, 300, 512, 768, 1024, 2048, 4096])
+@pytest.mark.parametrize("N", [300, 1024, 4096, 8192, 14336, 28672, 57344])
+def test_prefill_dispatch_does_not_depend_on_k(M, N):
+    routes = {w3a16_gemm_route(M, N, K, SMS) for K in (256, 1024, 4096, 8192, 28672, 65536)}
+    assert len(routes) == 1 and routes <= {"prefill", "prefill_ab"}, routes
 
 
 def test_route_depends_on_the_sm_count():

@@ -345,21 +345,27 @@ w3_status launch_prefill(const uint16_t *x, const int32_t *packed, const uint16_
     return cudaLaunchKernelEx(&cfg, prefill::prefill_kernel, prm) == cudaSuccess ? W3_OK : W3_ERR_CUDA;
 }
 
-// Which prefill kernel: both are paced by full waves of CTAs.  A wave of the shared-memory
-// kernel takes about 43 + 0.27 * BN us at K = 8192 (its dequantizing producers do not speed up
-// in proportion to a smaller tile), a wave of the tensor-memory kernel (256 x rows per tile)
-// about 55 us (measured on B200 over gate/down/q-shaped problems); the shared-memory kernel is
-// kept unless the other is predicted 2 % faster, and below 256 rows of x, where its CTA time
-// does not shrink with the batch.
+// Which prefill kernel.  Both run one CTA per SM and stream K in 64-wide stages, so each takes
+// (waves of CTAs) x (K / 64 stages) x (time of one stage of a wave), and only the stage times
+// differ.  Measured on B200 over 55 shapes (M 17..4096, N 300..57344, K 1152..28672; each
+// kernel timed alone), a wave's stage takes about
+//   prefill_kernel:    441 ns + 1.82 ns x BN x h   (BN rows of W per CTA; h = the share of its
+//                      two 128-row MMA tiles that hold rows of x; its dequantizing producers
+//                      set the fixed part, the MMAs' shared-memory operand reads the rest)
+//   prefill_ab_kernel: 313 ns + 0.51 ns x bn       (bn rows of x per CTA, 128 rows of W)
+// The K / 64 factor is common, so the choice holds for every K.  On those shapes the rule picks
+// the faster kernel to within 2.2 % (it is within 0.6 % on 19 shapes timed on another box); the
+// kernels are within a few per cent of each other at the shapes where it errs.
 bool prefer_prefill_ab(int M, int N, int sms) {
-    if (M < prefill_ab::kMaxBN) return false;
     const prefill::LaunchPlan po = prefill::plan(M, N, sms);
     const prefill_ab::LaunchPlan pa = prefill_ab::plan(M, N);
-    const double waves_o = std::ceil(static_cast<double>(po.grid.x) * po.grid.y / sms);
+    const int mt = (M + prefill::kTileM - 1) / prefill::kTileM;
+    const double h = static_cast<double>((M + prefill::kUmmaM - 1) / prefill::kUmmaM) / (2.0 * mt);
+    const double waves_o = std::ceil(static_cast<double>(po.grid.x) / sms);
     const double waves_a = std::ceil(static_cast<double>(pa.grid.x) / sms);
-    const double cost_o = waves_o * (43.0 + 0.27 * po.tile_n);
-    const double cost_a = waves_a * 55.0;
-    return cost_a < 0.98 * cost_o;
+    const double stage_o = 441.0 + 1.82 * po.tile_n * h;
+    const double stage_a = 313.0 + 0.51 * pa.bn;
+    return waves_a * stage_a < waves_o * stage_o;
 }
 
 // Prefill with the weights in tensor memory (prefill_swab.cuh).
@@ -586,9 +592,17 @@ enum class Route {
     Passes,         // no prefill kernel fits (K < 256): 16-row passes of the decode routes
 };
 
+// Whether the split decode has a launch plan (shared memory for the prepared x of a K slice,
+// a ring and the cluster's partial sums); the answer does not depend on the device's occupancy.
+bool split_fits(int64_t mb, int64_t N, int64_t K, int sms) {
+    return dsplit::plan(static_cast<int>(mb), static_cast<int>(N), static_cast<int>(K), sms,
+                        [](int, int) { return 0; })
+        .ok;
+}
+
 // The route of one pass of at most 16 batch rows.
 Route decode_route(int64_t mb, int64_t N, int64_t K, int sms) {
-    if (N >= dsplit::kBlockRows && mb >= kSplitMinBatch) return Route::DecodeSplit;
+    if (N >= dsplit::kBlockRows && mb >= kSplitMinBatch && split_fits(mb, N, K, sms)) return Route::DecodeSplit;
     if (N >= static_cast<int64_t>(decode_sk::kBlockRows) * sms &&
         decode_sk::applicable(static_cast<int>(mb), static_cast<int>(N), static_cast<int>(K)))
         return Route::DecodeStreamK;
@@ -697,9 +711,9 @@ w3_status run_gemm(const uint16_t *x, const int32_t *packed, const uint16_t *sca
         uint16_t *yp = y + m0 * N;
         switch (decode_route(mb, N, K, sms)) {
             case Route::DecodeSplit: {
+                // the route was chosen because a plan exists, with or without the occupancy answer
                 const dsplit::LaunchPlan sp = split_plan(mb, n, k, sms);
-                status = sp.ok ? launch_decode_split(xp, packed, scales, yp, mb, n, k, sp, st)
-                               : launch_decode(xp, packed, scales, yp, mb, n, k, sms, st);
+                status = sp.ok ? launch_decode_split(xp, packed, scales, yp, mb, n, k, sp, st) : W3_ERR_UNSUPPORTED;
                 break;
             }
             case Route::DecodeStreamK: status = launch_decode_sk(xp, packed, scales, yp, mb, n, k, sms, st); break;

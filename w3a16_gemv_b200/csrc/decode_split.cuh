@@ -476,7 +476,10 @@ inline int fitting_depth(int gs, int mt, int nb, int C) {
 }
 
 // Clusters of C CTAs that are resident at once; `active_clusters(C, smem)` asks the
-// device (occupancy query) and returns 0 when it cannot say.
+// device (occupancy query) and returns 0 when it cannot say.  Whether a plan exists does
+// not depend on that answer (the route query asks without a device): when fewer clusters
+// are resident than SMs / C and their larger share of blocks would not fit in shared
+// memory, the clusters run in waves instead.
 template <class ActiveClusters>
 inline LaunchPlan plan(int M, int N, int K, int num_sms, ActiveClusters active_clusters) {
     LaunchPlan best{};
@@ -486,32 +489,32 @@ inline LaunchPlan plan(int M, int N, int K, int num_sms, ActiveClusters active_c
     const int G = K / kGroup;
     const int NB = (N + kBlockRows - 1) / kBlockRows;
     int64_t best_cost = -1;
-    for (int C = 1; C <= kMaxCluster; C *= 2) {
-        if (C > G) break;
+    for (int C = 1; C <= kMaxCluster && C <= G; C *= 2) {
         const int gs = (G + C - 1) / C;
-        int ncl = num_sms / C;
-        for (int pass = 0; pass < 2 && ncl > 0; ++pass) {
-            const int nb = (NB + ncl - 1) / ncl;
-            const int depth = fitting_depth(gs, mt, nb, C);
-            if (depth == 0) {
-                ncl = 0;
-                break;
-            }
-            if (C == 1) break;
+        int ncl = num_sms / C < NB ? num_sms / C : NB;
+        if (ncl <= 0) break;
+        int nb = (NB + ncl - 1) / ncl;
+        int depth = fitting_depth(gs, mt, nb, C);
+        if (depth == 0) continue;
+        int waves = 1;
+        for (int pass = 0; C > 1 && pass < 2; ++pass) {
             const int fit = active_clusters(C, smem_layout(gs, mt, depth, nb, C).total);
             if (fit <= 0 || fit >= ncl) break;
-            ncl = fit;  // fewer clusters fit than SMs / C: plan for those
+            const int nb_fit = (NB + fit - 1) / fit;
+            const int depth_fit = fitting_depth(gs, mt, nb_fit, C);
+            if (depth_fit == 0) {
+                waves = (ncl + fit - 1) / fit;
+                break;
+            }
+            ncl = fit;  // plan for the clusters that are resident at once
+            nb = nb_fit;
+            depth = depth_fit;
         }
-        if (ncl <= 0) continue;
-        if (ncl > NB) ncl = NB;
-        const int nb = (NB + ncl - 1) / ncl;
-        const int depth = fitting_depth(gs, mt, nb, C);
-        if (depth == 0) continue;
         // The slowest CTA's (block, group) units, plus the cluster reduction.  The kernel streams
         // from HBM: CTAs with less work finish early and leave their bandwidth to the others, so
         // a finer split pays only when it gives many more SMs work (small N) or when x' of the
         // whole K range does not fit; a cluster costs about an eighth of the work.
-        const int64_t cost = static_cast<int64_t>(nb) * gs * 16 * (C > 1 ? 9 : 8) / 8;
+        const int64_t cost = static_cast<int64_t>(waves) * nb * gs * 16 * (C > 1 ? 9 : 8) / 8;
         if (best_cost < 0 || cost < best_cost) {
             best_cost = cost;
             best.ok = true;

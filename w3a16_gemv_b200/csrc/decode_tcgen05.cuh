@@ -140,6 +140,29 @@ struct FixupParams {
 // First unit of CTA c: the ranges [unit_begin(c), unit_begin(c + 1)) tile the units.
 __host__ __device__ inline int64_t unit_begin(int c, int64_t U, int P) { return static_cast<int64_t>(c) * U / P; }
 
+// A tile that several CTAs' ranges share is left as fp32 partial sums, two slots per CTA: slot 0
+// holds the first tile of CTA c's range, slot 1 its last (a range is contiguous, so no other
+// tile of it can be shared).
+__host__ __device__ inline int partial_slot(int c, int64_t t, int64_t U, int P, int G) {
+    return unit_begin(c, U, P) / G == t ? 0 : 1;
+}
+
+// The shared tile that fix-up block b finishes, or -1: the tile that the boundary
+// unit_begin(b + 1) cuts, unless that boundary is a tile boundary or an earlier boundary cuts
+// the same tile (an earlier block finishes it then).
+__host__ __device__ inline int64_t fixup_tile(int b, int64_t U, int P, int G) {
+    const int64_t u = unit_begin(b + 1, U, P);
+    const int64_t t0 = (u / G) * G;
+    if (u == t0 || unit_begin(b, U, P) > t0) return -1;
+    return u / G;
+}
+
+// Whether CTA c holds a part of tile t, for c at or after the block that finishes t: the CTAs
+// b, b + 1, ... up to the first one whose range starts after the tile.
+__host__ __device__ inline bool holds_part(int c, int64_t t, int64_t U, int P, int G) {
+    return c < P && unit_begin(c, U, P) < (t + 1) * G;
+}
+
 // ---- compile-time constants of the pair schedule ----------------------------------
 
 // bf16x2 (2^-e_lo, 2^-e_hi) for pair i: the scaling of x' in the pair's two slots.
@@ -311,10 +334,11 @@ __device__ __forceinline__ void permute_x(uint8_t *xs, int ns, int lane) {
 struct Walk {
     int64_t u, end;
     int G;
-    __device__ explicit Walk(const Params &p)
-        : u(unit_begin(blockIdx.x, p.U, p.P)), end(unit_begin(blockIdx.x + 1, p.U, p.P)), G(p.G) {}
+    __host__ __device__ Walk(int c, int64_t U, int P, int G_)
+        : u(unit_begin(c, U, P)), end(unit_begin(c + 1, U, P)), G(G_) {}
+    __device__ explicit Walk(const Params &p) : Walk(blockIdx.x, p.U, p.P, p.G) {}
     // next segment: tile t, first group g0, length len; false when done
-    __device__ bool next(int64_t &t, int &g0, int &len) {
+    __host__ __device__ bool next(int64_t &t, int &g0, int &len) {
         if (u >= end) return false;
         t = u / G;
         g0 = static_cast<int>(u - t * G);
@@ -508,7 +532,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_tc_kernel(const _
 
         Walk walk(p);
         int64_t t;
-        int g0, len, stage = 0, j = 0, seg = 0;
+        int g0, len, stage = 0, j = 0;
         while (ok && walk.next(t, g0, len)) {
 #pragma unroll
             for (int b = 0; b < kBatch; ++b) acc[b] = 0.f;
@@ -573,12 +597,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_tc_kernel(const _
                         if (b < p.M) p.y[static_cast<int64_t>(b) * p.N + n] = f32_to_bf16_rn(acc[b]);
                 }
             } else {  // shared tile: fp32 partial sums for the fix-up kernel
-                float *dst = p.partial + (static_cast<int64_t>(blockIdx.x) * 2 + (seg == 0 ? 0 : 1)) * kBatch * kRows + r;
+                float *dst = p.partial +
+                             (static_cast<int64_t>(blockIdx.x) * 2 + partial_slot(blockIdx.x, t, p.U, p.P, p.G)) *
+                                 kBatch * kRows +
+                             r;
 #pragma unroll
                 for (int b = 0; b < kBatch; ++b)
                     if (b < p.M) dst[b * kRows] = acc[b];
             }
-            ++seg;
         }
     }
 
@@ -595,11 +621,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_tc_kernel(const _
 // partial sums of the CTAs that cover it, in CTA order.
 __global__ void __launch_bounds__(kRows) decode_tc_fixup_kernel(const __grid_constant__ FixupParams p) {
     pdl_wait();
-    const int i = blockIdx.x + 1;
-    const int64_t u = unit_begin(i, p.U, p.P);
-    const int64_t t = u / p.G;
-    const int64_t t0 = t * p.G, t1 = t0 + p.G;
-    if (u == t0 || unit_begin(i - 1, p.U, p.P) > t0) return;
+    const int64_t t = fixup_tile(blockIdx.x, p.U, p.P, p.G);
+    if (t < 0) return;
     const int r = threadIdx.x;
     const int64_t n = t * kRows + r;
     if (n >= p.N) return;
@@ -608,15 +631,11 @@ __global__ void __launch_bounds__(kRows) decode_tc_fixup_kernel(const __grid_con
     for (int b = 0; b < kBatch; ++b) acc[b] = 0.f;
     // contributors in rounds of 4 whose loads are all issued before the adds
     constexpr int kRound = 4;
-    for (int c = i - 1; c < p.P;) {
+    for (int c = blockIdx.x; c < p.P;) {
         const float *src[kRound];
         int cnt = 0;
-        for (; cnt < kRound && c < p.P; ++c) {
-            const int64_t uc = unit_begin(c, p.U, p.P);
-            if (uc >= t1) break;
-            const int slot = (uc / p.G == t) ? 0 : 1;
-            src[cnt++] = p.partial + (static_cast<int64_t>(c) * 2 + slot) * kBatch * kRows + r;
-        }
+        for (; cnt < kRound && holds_part(c, t, p.U, p.P, p.G); ++c)
+            src[cnt++] = p.partial + (static_cast<int64_t>(c) * 2 + partial_slot(c, t, p.U, p.P, p.G)) * kBatch * kRows + r;
         float v[kRound][kBatch];
 #pragma unroll
         for (int q = 0; q < kRound; ++q)

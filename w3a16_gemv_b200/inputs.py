@@ -145,7 +145,15 @@ def workloads() -> dict[str, Workload]:
                                               "absnormal", "normal_outliers")
     for name, n, k in LLAMA70B_LAYER:
         w[f"layer_{name}_m1"] = Workload(f"layer_{name}_m1", 1, n, k, "uniform8", "lognormal")
+    # mid-size batches on gate_proj and q_proj: the 32-wide tensor-core decode (M = 24) and
+    # both prefill kernels (the dispatch picks per shape)
+    for m in (24, 33, 64, 128, 160, 255):
+        w[f"mid_gate_28672x8192_m{m}"] = Workload(f"mid_gate_28672x8192_m{m}", m, 28672, 8192, "uniform8",
+                                                  "lognormal")
+    w["mid_q_8192x8192_m64"] = Workload("mid_q_8192x8192_m64", 64, 8192, 8192, "gsq_5level", "absnormal",
+                                        "normal_outliers")
     w["prefill_2048x28672x8192"] = Workload("prefill_2048x28672x8192", 2048, 28672, 8192, "uniform8", "lognormal")
-    # a batch at which the tensor-memory prefill kernel is the one launched
+    # batches at which each prefill kernel is the one launched
     w["prefill_1024x28672x8192"] = Workload("prefill_1024x28672x8192", 1024, 28672, 8192, "uniform8", "lognormal")
+    w["prefill_512x28672x8192"] = Workload("prefill_512x28672x8192", 512, 28672, 8192, "uniform8", "lognormal")
     return w
