@@ -290,15 +290,10 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(const __gr
         return n;
     }();
 
-    // stream weights before preparing x (the weights never come from the previous kernel)
     int64_t ibl = blk0;
     int ig = g_first0;
     int issued = 0;
     int issue_slot = 0;  // == issued % depth
-    for (; issued < depth - 1 && issued < nstages_total; ++issued) {
-        advance(ibl, ig, issue(ibl, ig, issue_slot));
-        issue_slot = (issue_slot + 1 == depth) ? 0 : issue_slot + 1;
-    }
     // x (and, at the end, y) may belong to the previous kernel in the stream
     pdl_wait();
     decode::Params dp;  // prepare_x reads x, M and K only
@@ -320,6 +315,14 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(const __gr
             nq[it] = make_float4(a, b, a, b);
         }
         __syncthreads();
+    }
+    // The first weight stages are issued only now.  Issued before x is prepared, their copies
+    // slow the CTA's loads of x, the main loop starts later, and a call takes longer: 47.4 against
+    // 45.1 us at M = 16 and 33.3 against 31.5 us at M = 8 on gate_proj.  (The stream-K decode,
+    // whose x is a quarter of the size or less, gains from issuing them first.)
+    for (; issued < depth - 1 && issued < nstages_total; ++issued) {
+        advance(ibl, ig, issue(ibl, ig, issue_slot));
+        issue_slot = (issue_slot + 1 == depth) ? 0 : issue_slot + 1;
     }
 
     // B fragments: lanes whose batch row is >= MT read words of other rows; the MMA keeps
