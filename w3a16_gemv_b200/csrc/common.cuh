@@ -158,6 +158,11 @@ __device__ __forceinline__ float4 ld_dsmem_f4(uint32_t addr) {
     return v;
 }
 
+__device__ __forceinline__ void st_dsmem_f4(uint32_t addr, const float4 &v) {
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
+                 : "memory");
+}
+
 // ---- bit manipulation ----------------------------------------------------------------
 
 // (a & MASK) | c in exactly one LOP3: the mask is the instruction's immediate

@@ -13,10 +13,12 @@
 // per SM would.  Inside a CTA the (block, group) units of the slice are cut
 // into equal contiguous ranges, one per warp ("stream-K"): a warp's range is
 // the end of one block, whole blocks and the start of another.  Blocks split
-// between warps are added in warp order through shared memory; with C > 1
-// every CTA then holds the partial sums of all the cluster's blocks over its
-// slice, and rank q adds the C slices of its share of the blocks in rank order
-// through distributed shared memory.  Every sum has a fixed order: results are
+// between warps are added in warp order through shared memory.  With C > 1 the
+// blocks of a cluster are shared out among its ranks; as a CTA finishes a
+// block's sum over its slice it stores it into the shared memory of the rank
+// that owns the block (distributed shared memory, during the main loop), and
+// after one cluster barrier each rank adds the C slices of its blocks in rank
+// order from its own shared memory.  Every sum has a fixed order: results are
 // deterministic, and no global scratch or atomic is used.
 //
 // Loads: each warp streams its range through a private ring of tiled TMA
@@ -56,6 +58,10 @@ struct SmemLayout {
     int xs_off, corr_off, cpart_off, ncorr_off, bar_off, ring_off, slot_off, pb_off, total;
 };
 
+// Blocks a rank of a C-CTA cluster owns for the final sum, at most: rank q owns the cluster's
+// blocks [nb*q/C, nb*(q+1)/C).
+__host__ __device__ constexpr int share_blocks(int nb, int C) { return (nb + C - 1) / C; }
+
 // gs: groups of the CTA's K slice (at most); nb: blocks of a cluster (at most).
 __host__ __device__ inline SmemLayout smem_layout(int gs, int mt, int depth, int nb, int C) {
     const int nt = n_tiles(mt);
@@ -67,8 +73,8 @@ __host__ __device__ inline SmemLayout smem_layout(int gs, int mt, int depth, int
     L.bar_off = decode::align_up(L.ncorr_off + gs * nt * 4 * 16, 16);      // u64 [warps][depth]
     L.ring_off = decode::align_up(L.bar_off + kWarps * depth * 8, 128);    // [warps][depth][stage bytes]
     L.slot_off = L.ring_off + kWarps * depth * stage_bytes(mt);            // float4 [warps][2 tiles][nt][32]
-    L.pb_off = L.slot_off + kWarps * 2 * nt * 32 * 16;                     // float4 [nb][2 tiles][nt][32] (C > 1)
-    L.total = L.pb_off + (C > 1 ? nb * 2 * nt * 32 * 16 : 0);
+    L.pb_off = L.slot_off + kWarps * 2 * nt * 32 * 16;                     // float4 [C][share][2 tiles][nt][32] (C > 1)
+    L.total = L.pb_off + (C > 1 ? C * share_blocks(nb, C) * 2 * nt * 32 * 16 : 0);
     return L;
 }
 
@@ -332,15 +338,26 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(const __gr
     float4 *park = reinterpret_cast<float4 *>(smem + L.slot_off) + warp * 2 * NT * 32;
     float4 *pb = reinterpret_cast<float4 *>(smem + L.pb_off);
 
-    // a block's sums over the CTA's slice: to y (C == 1) or to the cluster's partial buffer
+    // a block's sums over the CTA's slice: to y (C == 1), or into slot [q] of the block in the
+    // shared memory of the rank that owns it
+    const int nbc = b_end - b_begin;
+    const int share = share_blocks(p.nb_max, C);
     auto emit = [&](int block, const float (&v)[2][NT][4]) {
+        const int lb = block - b_begin;
+        int qo = 0;  // owner rank: lb in [nbc*qo/C, nbc*(qo+1)/C)
+        while (qo + 1 < C && lb >= nbc * (qo + 1) / C) ++qo;
+        const int lo = lb - nbc * qo / C;
 #pragma unroll
         for (int t = 0; t < 2; ++t)
 #pragma unroll
             for (int u = 0; u < NT; ++u) {
                 const float4 f = make_float4(v[t][u][0], v[t][u][1], v[t][u][2], v[t][u][3]);
-                if (C == 1) store_frag(p.y, N, M, block, t, u, r, c, f);
-                else pb[(((block - b_begin) * 2 + t) * NT + u) * 32 + lane] = f;
+                if (C == 1) {
+                    store_frag(p.y, N, M, block, t, u, r, c, f);
+                } else {
+                    const uint32_t local = smem_addr(pb + ((((q * share + lo) * 2 + t) * NT + u) * 32 + lane));
+                    st_dsmem_f4(map_to_rank(local, qo), f);
+                }
             }
     };
 
@@ -443,26 +460,24 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(const __gr
     }
     if (C == 1) return;
 
-    // ---- the cluster: rank q adds the C slices of its share of the blocks, in rank order ----
-    __syncthreads();
-    cluster_sync();  // every CTA's partial buffer is complete
-    const int nb = b_end - b_begin;
-    const int sb0 = nb * q / C, sb1 = nb * (q + 1) / C;
+    // ---- the cluster: rank q adds the C slices of its blocks, in rank order ----
+    // The barrier makes every rank's stores into this CTA's shared memory visible.  After it no
+    // CTA touches another's shared memory, so a CTA may leave as soon as it is done.
+    cluster_sync();
+    const int sb0 = nbc * q / C, sb1 = nbc * (q + 1) / C;
     const int items = (sb1 - sb0) * 2 * NT * 32;
     for (int it = threadIdx.x; it < items; it += blockDim.x) {
-        const int ln = it & 31, u = (it >> 5) % NT, t = (it / (32 * NT)) & 1, lb = sb0 + it / (64 * NT);
-        const uint32_t local = smem_addr(pb + ((lb * 2 + t) * NT + u) * 32 + ln);
-        float4 v = ld_dsmem_f4(map_to_rank(local, 0));
+        const int ln = it & 31, u = (it >> 5) % NT, t = (it / (32 * NT)) & 1, lo = it / (64 * NT);
+        float4 v = pb[((lo * 2 + t) * NT + u) * 32 + ln];
         for (int rk = 1; rk < C; ++rk) {
-            const float4 f = ld_dsmem_f4(map_to_rank(local, rk));
+            const float4 f = pb[(((rk * share + lo) * 2 + t) * NT + u) * 32 + ln];
             v.x += f.x;
             v.y += f.y;
             v.z += f.z;
             v.w += f.w;
         }
-        if (ok) store_frag(p.y, N, M, b_begin + lb, t, u, ln >> 2, ln & 3, v);
+        if (ok) store_frag(p.y, N, M, b_begin + sb0 + lo, t, u, ln >> 2, ln & 3, v);
     }
-    cluster_sync();  // no CTA leaves while another still reads its shared memory
 }
 
 struct LaunchPlan {
