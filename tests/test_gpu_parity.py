@@ -78,9 +78,12 @@ SMALL = [
     (129, 600, 512, "uniform8", "lognormal", "normal"),
 ]
 
-# (route, M, N, K, codes, scales, x): shapes the dispatch sends to a given prefill kernel
-# (asserted with w3a16_gemm_route), checked in full.
+# (route, M, N, K, codes, scales, x): shapes the dispatch sends to a given kernel (asserted with
+# w3a16_gemm_route), checked in full.
 ROUTED = [
+    # 2..4 batch rows over a K too tall for the stream-K decode's prepared x: the split decode
+    ("decode_split", 4, 4800, 12416, "uniform8", "lognormal", "normal"),
+    ("decode_split", 2, 4800, 24704, "gsq_5level", "absnormal", "normal_outliers"),
     # the shared-memory prefill: one 128-row MMA tile of x; a ragged second one; a ragged third
     # 256-row batch tile; four batch tiles; ragged last W tiles (N = 20001)
     ("prefill", 33, 20001, 256, "uniform8", "lognormal", "normal"),
@@ -109,7 +112,7 @@ def test_small_shapes_full_parity(orc, case):
 
 
 @pytest.mark.parametrize("case", ROUTED, ids=[f"{c[0]}_{_id(c[1:])}" for c in ROUTED])
-def test_prefill_routes_full_parity(orc, case):
+def test_routed_shapes_full_parity(orc, case):
     assert w3a16_gemm_route(*case[1:4]) == case[0]
     _full_parity(orc, case[1:])
 

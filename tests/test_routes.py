@@ -40,7 +40,9 @@ def test_every_shape_has_a_known_route(M, N, K):
         # cluster's partial sums; the older cluster decode otherwise
         assert r in (("decode_split", "decode") if N >= 32 else ("decode",))
     if M <= 4:
-        assert r in ("decode_sk", "decode")
+        assert r in ("decode_sk", "decode_split", "decode")
+        if r == "decode_split":  # many rows, x of the whole K range too large for the stream-K decode
+            assert N >= 32 * SMS and M * K * 2 > 96 * 1024
     if r == "decode_sk":
         assert M <= 4 and N >= 32 * SMS
     if r == "decode_tc32":
@@ -105,6 +107,16 @@ def test_prefill_dispatch_picks_the_measured_faster_kernel(shape):
 def test_prefill_dispatch_does_not_depend_on_k(M, N):
     routes = {w3a16_gemm_route(M, N, K, SMS) for K in (256, 1024, 4096, 8192, 28672, 65536)}
     assert len(routes) == 1 and routes <= {"prefill", "prefill_ab"}, routes
+
+
+def test_tall_k_small_batches_take_the_split_decode():
+    # down_proj at 2..4 batch rows: the stream-K decode's prepared x of all of K does not fit
+    assert w3a16_gemm_route(1, 8192, 28672, SMS) == "decode_sk"
+    for M in (2, 3, 4):
+        assert w3a16_gemm_route(M, 8192, 28672, SMS) == "decode_split"
+    assert w3a16_gemm_route(4, 28672, 8192, SMS) == "decode_sk"
+    # few rows: the older decode keeps the small shapes
+    assert w3a16_gemm_route(4, 1024, 28672, SMS) == "decode"
 
 
 def test_route_depends_on_the_sm_count():

@@ -586,7 +586,7 @@ w3_status launch_decode_split(const uint16_t *x, const int32_t *packed, const ui
 constexpr int kSplitMinBatch = 5;
 
 enum class Route {
-    DecodeSplit,    // decode_split_kernel: M <= 16, N >= 32 (cluster split-K, mma.sync)
+    DecodeSplit,    // decode_split_kernel: 5 <= M <= 16 (and tall K at M <= 4), cluster split-K, mma.sync
     DecodeStreamK,  // decode_sk_kernel: M <= 4, at least one 32-row block per SM
     Decode,         // decode_kernel: the remaining small shapes (M <= 16)
     DecodeTc32,     // decode_tc32 decode_tc_kernel (+ fix-up): 17 <= M <= 32, N >= 256
@@ -606,9 +606,13 @@ bool split_fits(int64_t mb, int64_t N, int64_t K, int sms) {
 // The route of one pass of at most 16 batch rows.
 Route decode_route(int64_t mb, int64_t N, int64_t K, int sms) {
     if (N >= dsplit::kBlockRows && mb >= kSplitMinBatch && split_fits(mb, N, K, sms)) return Route::DecodeSplit;
-    if (N >= static_cast<int64_t>(decode_sk::kBlockRows) * sms &&
-        decode_sk::applicable(static_cast<int>(mb), static_cast<int>(N), static_cast<int>(K)))
-        return Route::DecodeStreamK;
+    if (N >= static_cast<int64_t>(decode_sk::kBlockRows) * sms) {
+        if (decode_sk::applicable(static_cast<int>(mb), static_cast<int>(N), static_cast<int>(K)))
+            return Route::DecodeStreamK;
+        // many rows, but the prepared x of the whole K range does not fit (a tall K at 2..4 batch
+        // rows): the split decode prepares x for a K slice only
+        if (split_fits(mb, N, K, sms)) return Route::DecodeSplit;
+    }
     return Route::Decode;
 }
 
