@@ -439,20 +439,39 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(const __gr
         if (own_u >= u0 && own_u + Gs > u1) {
             const int block = b_begin + static_cast<int>(own_u / Gs);
             const float4 *all = reinterpret_cast<const float4 *>(smem + L.slot_off);
-            for (int w2 = warp + 1; w2 < kWarps; ++w2) {
-                int64_t a0, a1;
-                warp_range(units, w2, kWarps, a0, a1);
-                if (a0 >= own_u + Gs) break;
-                if (a1 <= a0) continue;
+            // The later warps whose range starts inside the block, in warp order.  Warp starts
+            // increase with the warp, so "starts before the block ends" selects a run of warps.
+            // Four warps' parts are loaded before any is added (the loads overlap; the adds keep
+            // warp order).  32-bit unit arithmetic: a CTA has fewer than 2^32 / kWarps units.
+            const uint32_t units32 = static_cast<uint32_t>(units), own_end = static_cast<uint32_t>(own_u + Gs);
 #pragma unroll
-                for (int t = 0; t < 2; ++t)
+            for (int wc = 1; wc < kWarps; wc += 4) {
+                float4 f[4][2][NT];
+                bool use[4];
 #pragma unroll
-                    for (int u = 0; u < NT; ++u) {
-                        const float4 f = all[(w2 * 2 * NT + t * NT + u) * 32 + lane];
-                        acc[t][u][0] += f.x;
-                        acc[t][u][1] += f.y;
-                        acc[t][u][2] += f.z;
-                        acc[t][u][3] += f.w;
+                for (int i = 0; i < 4; ++i) {
+                    const int w2 = wc + i;
+                    const uint32_t a0 = units32 * static_cast<uint32_t>(w2) / kWarps;
+                    const uint32_t a1 = units32 * static_cast<uint32_t>(w2 + 1) / kWarps;
+                    use[i] = w2 < kWarps && w2 > warp && a0 < own_end && a1 > a0;
+#pragma unroll
+                    for (int t = 0; t < 2; ++t)
+#pragma unroll
+                        for (int u = 0; u < NT; ++u)
+                            f[i][t][u] = use[i] ? all[(w2 * 2 * NT + t * NT + u) * 32 + lane] : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    if (use[i]) {
+#pragma unroll
+                        for (int t = 0; t < 2; ++t)
+#pragma unroll
+                            for (int u = 0; u < NT; ++u) {
+                                acc[t][u][0] += f[i][t][u].x;
+                                acc[t][u][1] += f[i][t][u].y;
+                                acc[t][u][2] += f[i][t][u].z;
+                                acc[t][u][3] += f[i][t][u].w;
+                            }
                     }
             }
             emit(block, acc);
