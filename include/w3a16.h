@@ -205,12 +205,12 @@ w3_status w3a16_gemm_native(const uint16_t *x, const int32_t *native, const uint
 /*
  * w3a16_gemm_route -- which kernels w3a16_gemm (and w3a16_gemm_noalloc) run for
  * an M x N x K product on a GPU with `num_sms` SMs, as a short name:
+ *   "decode_sk"   persistent stream-K mma.sync decode (M <= 4, N >= 32 * num_sms,
+ *                 x of the whole K range fits in shared memory);
  *   "decode_split" mma.sync decode, K split over a thread-block cluster with a
- *                 fixed-order reduction in distributed shared memory
- *                 (5 <= M <= 16, N >= 32; and M <= 4 with N >= 32 * num_sms when
- *                 x of the whole K range is too large for "decode_sk");
- *   "decode_sk"   persistent stream-K mma.sync decode (M <= 4, N >= 32 * num_sms);
- *   "decode"      mma.sync decode with cluster split-K (the other M <= 16 shapes);
+ *                 fixed-order reduction in distributed shared memory (the other
+ *                 M <= 16 shapes with N >= 32 where its plan fits);
+ *   "decode"      mma.sync decode with cluster split-K (the remaining M <= 16 shapes);
  *   "decode_tc32" tensor-core (tcgen05) decode, 32 columns (17 <= M <= 32, N >= 256);
  *   "prefill"     tcgen05 GEMM, weights dequantized into shared memory;
  *   "prefill_ab"  tcgen05 GEMM, weights dequantized into tensor memory;

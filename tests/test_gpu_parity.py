@@ -198,7 +198,9 @@ def _probe(orc, M, N, K, seed):
 PROBES = [
     ("decode_sk", 1, 4800, 256),
     ("decode_sk", 4, 4800, 384),
-    ("decode", 1, 300, 256),
+    ("decode", 1, 20, 512),
+    ("decode_split", 1, 300, 256),
+    ("decode_split", 4, 1024, 1152),
     ("decode", 16, 20, 256),
     ("decode_split", 5, 300, 384),
     ("decode_split", 8, 1000, 256),

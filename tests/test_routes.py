@@ -41,8 +41,8 @@ def test_every_shape_has_a_known_route(M, N, K):
         assert r in (("decode_split", "decode") if N >= 32 else ("decode",))
     if M <= 4:
         assert r in ("decode_sk", "decode_split", "decode")
-        if r == "decode_split":  # many rows, x of the whole K range too large for the stream-K decode
-            assert N >= 32 * SMS and M * K * 2 > 96 * 1024
+    if r == "decode":  # fewer than 32 rows, or a split plan that does not fit (K above 8192 here)
+        assert N < 32 or K > 8192
     if r == "decode_sk":
         assert M <= 4 and N >= 32 * SMS
     if r == "decode_tc32":
@@ -62,8 +62,9 @@ def test_benchmarked_shapes():
     assert w3a16_gemm_route(16, 28672, 8192, SMS) == "decode_split"
     assert w3a16_gemm_route(24, 28672, 8192, SMS) == "decode_tc32"
     assert w3a16_gemm_route(2048, 28672, 8192, SMS) in ("prefill", "prefill_ab")
-    # fewer 32-row blocks than SMs at M <= 4: the mma.sync decode with cluster split-K
-    assert w3a16_gemm_route(1, 1024, 8192, SMS) == "decode"
+    # fewer 32-row blocks than SMs at M <= 4: the split decode; fewer than 32 rows: the older decode
+    assert w3a16_gemm_route(1, 1024, 8192, SMS) == "decode_split"
+    assert w3a16_gemm_route(1, 4096, 4096, SMS) == "decode_split"
     assert w3a16_gemm_route(8, 20, 8192, SMS) == "decode"
 
 
@@ -115,11 +116,10 @@ def test_tall_k_small_batches_take_the_split_decode():
     for M in (2, 3, 4):
         assert w3a16_gemm_route(M, 8192, 28672, SMS) == "decode_split"
     assert w3a16_gemm_route(4, 28672, 8192, SMS) == "decode_sk"
-    # few rows: the older decode keeps the small shapes
-    assert w3a16_gemm_route(4, 1024, 28672, SMS) == "decode"
+    assert w3a16_gemm_route(4, 1024, 28672, SMS) == "decode_split"
 
 
 def test_route_depends_on_the_sm_count():
     # the stream-K decode needs one 32-row block per SM
     assert w3a16_gemm_route(1, 4800, 1024, 148) == "decode_sk"
-    assert w3a16_gemm_route(1, 4800, 1024, 160) == "decode"
+    assert w3a16_gemm_route(1, 4800, 1024, 160) == "decode_split"
