@@ -186,67 +186,40 @@ struct Params {
 };
 
 // Prepare x' and the per-group corrections for groups [g0, g0 + ng) of the
-// CTA's range.  Batch rows M..MT-1 are zero.  An item is 32 consecutive k of one
-// row (four 16-byte loads).  Each thread loads kPrepBatch items before it
-// transforms them; `after_loads` runs once in every thread (warp-uniformly) right
-// after the first batch of loads is issued, so that work issued there (the
-// first weight copies) queues behind the loads of x instead of ahead of them.
-constexpr int kPrepBatch = 3;
-
-struct NoHook {
-    __device__ void operator()() const {}
-};
-
-template <int MT, class AfterLoads = NoHook>
-__device__ __forceinline__ void prepare_x(const Params &p, uint8_t *smem, const SmemLayout &L, int g0, int ng,
-                                          AfterLoads after_loads = AfterLoads()) {
+// CTA's range.  Batch rows M..MT-1 are zero.
+template <int MT>
+__device__ __forceinline__ void prepare_x(const Params &p, uint8_t *smem, const SmemLayout &L, int g0, int ng) {
     constexpr int NT = (MT + 7) / 8;
     uint32_t *xs = reinterpret_cast<uint32_t *>(smem + L.xs_off);
     float *corr = reinterpret_cast<float *>(smem + L.corr_off);
     float *cpart = reinterpret_cast<float *>(smem + L.cpart_off);
     const int items = ng * MT * 4;
-    const int step = kPrepBatch * static_cast<int>(blockDim.x);
-    for (int it0 = threadIdx.x, round = 0; round == 0 || it0 < items; it0 += step, ++round) {
-        uint4 raw[kPrepBatch][4];
+    for (int it = threadIdx.x; it < items; it += blockDim.x) {
+        const int c = it & 3;
+        const int m = (it >> 2) % MT;
+        const int g = it / (4 * MT);
+        uint4 raw[4] = {};
+        if (m < p.M) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(p.x + static_cast<int64_t>(m) * p.K +
+                                                               static_cast<int64_t>(g0 + g) * kGroup + 32 * c);
 #pragma unroll
-        for (int b = 0; b < kPrepBatch; ++b) {
-            const int it = it0 + b * blockDim.x;
-            const int c = it & 3;
-            const int m = (it >> 2) % MT;
-            const int g = it / (4 * MT);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) raw[b][i] = make_uint4(0u, 0u, 0u, 0u);
-            if (it < items && m < p.M) {
-                const uint4 *src = reinterpret_cast<const uint4 *>(p.x + static_cast<int64_t>(m) * p.K +
-                                                                   static_cast<int64_t>(g0 + g) * kGroup + 32 * c);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) raw[b][i] = __ldg(src + i);
-            }
+            for (int i = 0; i < 4; ++i) raw[i] = __ldg(src + i);
         }
-        if (round == 0) after_loads();
+        const uint16_t *xv = reinterpret_cast<const uint16_t *>(raw);
+        uint32_t *dst = xs + (((g * 8) * MT + m) * 4 + c) * 2;
 #pragma unroll
-        for (int b = 0; b < kPrepBatch; ++b) {
-            const int it = it0 + b * blockDim.x;
-            if (it >= items) break;
-            const int c = it & 3;
-            const int m = (it >> 2) % MT;
-            const int g = it / (4 * MT);
-            const uint16_t *xv = reinterpret_cast<const uint16_t *>(raw[b]);
-            uint32_t *dst = xs + (((g * 8) * MT + m) * 4 + c) * 2;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const PairSpec ps = pair_spec(i);
-                // uint2 index ((g*8 + t)*MT + m)*4 + c, component i&1, t = i/2
-                dst[(i >> 1) * MT * 8 + (i & 1)] =
-                    scaled_bf16(xv[ps.lo], ps.elo) | (scaled_bf16(xv[ps.hi], ps.ehi) << 16);
-            }
-            // corr partial, positions in ascending order for a fixed summation order
-            float part = 0.f;
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-                part = fmaf(128.0f / static_cast<float>(1 << code_shift(j)) + 4.0f, bf16_bits_to_f32(xv[j]), part);
-            cpart[(g * MT + m) * 4 + c] = part;
+        for (int i = 0; i < 16; ++i) {
+            const PairSpec ps = pair_spec(i);
+            // uint2 index ((g*8 + t)*MT + m)*4 + c, component i&1, t = i/2
+            dst[(i >> 1) * MT * 8 + (i & 1)] =
+                scaled_bf16(xv[ps.lo], ps.elo) | (scaled_bf16(xv[ps.hi], ps.ehi) << 16);
         }
+        // corr partial, positions in ascending order for a fixed summation order
+        float part = 0.f;
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            part = fmaf(128.0f / static_cast<float>(1 << code_shift(j)) + 4.0f, bf16_bits_to_f32(xv[j]), part);
+        cpart[(g * MT + m) * 4 + c] = part;
     }
     __syncthreads();
     for (int it = threadIdx.x; it < ng * 8 * NT; it += blockDim.x) {

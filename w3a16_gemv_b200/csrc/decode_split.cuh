@@ -310,16 +310,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(const __gr
     dl.xs_off = L.xs_off;
     dl.corr_off = L.corr_off;
     dl.cpart_off = L.cpart_off;
-    // The first weight stages are issued right after this CTA's loads of x: issued before them,
-    // their copies delay x (and the start of the main loop); issued after x is prepared, the
-    // first stage's DRAM latency is not hidden.
-    auto prologue = [&] {
-        for (; issued < depth - 1 && issued < nstages_total; ++issued) {
-            advance(ibl, ig, issue(ibl, ig, issue_slot));
-            issue_slot = (issue_slot + 1 == depth) ? 0 : issue_slot + 1;
-        }
-    };
-    decode::prepare_x<MT>(dp, smem, dl, gq0, Gs, prologue);
+    decode::prepare_x<MT>(dp, smem, dl, gq0, Gs);
     // each MMA chain starts from -corr: (-corr[8u+2c], -corr[8u+2c+1]) for rows r and r+8
     {
         const float *cf = reinterpret_cast<const float *>(smem + L.corr_off);
@@ -330,6 +321,14 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(const __gr
             nq[it] = make_float4(a, b, a, b);
         }
         __syncthreads();
+    }
+    // The first weight stages are issued only now.  Issued before x is prepared, their copies
+    // slow the CTA's loads of x, the main loop starts later, and a call takes longer: 47.4 against
+    // 45.1 us at M = 16 and 33.3 against 31.5 us at M = 8 on gate_proj.  (The stream-K decode,
+    // whose x is a quarter of the size or less, gains from issuing them first.)
+    for (; issued < depth - 1 && issued < nstages_total; ++issued) {
+        advance(ibl, ig, issue(ibl, ig, issue_slot));
+        issue_slot = (issue_slot + 1 == depth) ? 0 : issue_slot + 1;
     }
 
     // B fragments: lanes whose batch row is >= MT read words of other rows; the MMA keeps
