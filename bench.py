@@ -853,8 +853,9 @@ def run_gpu(args):
         "roofline": roofline,
         "e2e": e2e,
         "gpu_launches": args.steps * sum(kernels_per_call(m, N_ROWS, K_COLS, sms) for m in BATCHES),
-        "per_call_timing": f"calls[]: CUDA events around each call over {brk_steps} further steps (no overlap "
-                           "between calls); value: the K steps back to back",
+        "per_call_timing": f"calls[].us_mean: each call launched {brk_steps} times back to back (rotating weight "
+                           "copies, programmatic dependent launch), CUDA events around the run; us_isolated_*: "
+                           "an event pair around every call; value: the K steps back to back",
         "clocks": clocks,
     }
     del packs, scales, x_all, xs, ys, x_dev, y_dev
