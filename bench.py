@@ -80,10 +80,12 @@ def kernel_name(M: int, N: int, K: int, sms: int) -> str:
 
 
 def kernels_per_call(M: int, N: int, K: int, sms: int) -> int:
-    """Kernels one w3a16_gemm call launches: the 32-wide tensor-core decode is followed by its
-    partial-sum fix-up kernel when the work is split over more than one CTA (always, at these
-    sizes); every other route is one kernel."""
-    return 2 if route(M, N, K, sms) == "decode_tc32" else 1
+    """Kernels one w3a16_gemm call launches (asked from the library): the 32-wide tensor-core
+    decode is followed by a fix-up kernel when CTA boundaries split its row tiles; every other
+    route is one kernel (one per 16-row pass for the passes route)."""
+    from w3a16_gemv_b200 import w3a16_gemm_launches
+
+    return w3a16_gemm_launches(M, N, K, num_sms=sms)
 
 
 def step_bytes() -> int:

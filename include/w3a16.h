@@ -224,6 +224,15 @@ w3_status w3a16_gemm_native(const uint16_t *x, const int32_t *native, const uint
 const char *w3a16_gemm_route(int64_t M, int64_t N, int64_t K, int32_t num_sms);
 
 /*
+ * w3a16_gemm_launches -- how many kernels one w3a16_gemm (or w3a16_gemm_noalloc)
+ * call launches for an M x N x K product on a GPU with `num_sms` SMs: 2 where
+ * the tensor-core decode ("decode_tc32") splits row tiles between CTAs and a
+ * fix-up kernel finishes them, one per 16-row pass for "passes", 1 for every
+ * other route.  Host only, like w3a16_gemm_route; -1 where that returns NULL.
+ */
+int32_t w3a16_gemm_launches(int64_t M, int64_t N, int64_t K, int32_t num_sms);
+
+/*
  * w3_check_device_error -- synchronise `stream`, then report and clear the
  * current device's error flag: W3_OK, or W3_ERR_TIMEOUT if a kernel of this
  * library gave up a bounded wait since the last check.  W3_ERR_CUDA if the

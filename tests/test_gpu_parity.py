@@ -198,7 +198,7 @@ def _probe(orc, M, N, K, seed):
 PROBES = [
     ("decode_sk", 1, 4800, 256),
     ("decode_sk", 4, 4800, 384),
-    ("decode_sk", 1, 4768, 1152),   # paired CTAs: 149 blocks over 28 CTAs
+    ("decode_sk", 1, 4768, 1152),   # 149 blocks over 28 CTAs (5 or 6 each), split between warps
     ("decode", 1, 20, 512),
     ("decode_split", 1, 300, 256),
     ("decode_split", 4, 1024, 1152),

@@ -2,12 +2,12 @@
 
 w3a16_gemm_route depends only on the shape and the SM count, so the dispatch
 rules can be checked on the host: which kernel serves each batch size of the
-benchmarked shapes, the batch-size boundaries between routes, and that invalid
-shapes have no route.
+benchmarked shapes, the batch-size boundaries between routes, how many kernels
+a call launches, and that invalid shapes have no route.
 """
 import pytest
 
-from w3a16_gemv_b200 import _binding, build, w3a16_gemm_route
+from w3a16_gemv_b200 import _binding, build, w3a16_gemm_launches, w3a16_gemm_route
 
 SMS = 148  # B200
 
@@ -123,3 +123,18 @@ def test_route_depends_on_the_sm_count():
     # the stream-K decode needs one 32-row block per SM
     assert w3a16_gemm_route(1, 4800, 1024, 148) == "decode_sk"
     assert w3a16_gemm_route(1, 4800, 1024, 160) == "decode_split"
+
+
+def test_kernels_per_call():
+    """One kernel per call, plus the fix-up kernel where the tensor-core decode splits row tiles
+    between CTAs, and one per 16-row pass."""
+    f = w3a16_gemm_launches
+    assert f(1, 28672, 8192, SMS) == 1 and f(4, 28672, 8192, SMS) == 1  # stream-K decode
+    assert f(16, 28672, 8192, SMS) == 1  # split decode
+    assert f(24, 28672, 8192, SMS) == 2  # tensor-core decode and its fix-up
+    assert f(64, 28672, 8192, SMS) == 1 and f(2048, 28672, 8192, SMS) == 1  # prefill kernels
+    # passes: M = 36 with K = 128 is two 16-row passes and one 4-row pass
+    assert w3a16_gemm_route(36, 28672, 128, num_sms=SMS) == "passes"
+    assert f(36, 28672, 128, SMS) == 3
+    for args in ((0, 16, 128, SMS), (1, 0, 128, SMS), (1, 16, 192, SMS), (1, 16, 128, 0)):
+        assert _binding.lib().w3a16_gemm_launches(*args) == -1

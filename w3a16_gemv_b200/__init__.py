@@ -26,6 +26,7 @@ from ._binding import (  # noqa: F401
     w3a16_gemm,
     w3a16_gemm_native,
     w3a16_gemm_noalloc,
+    w3a16_gemm_launches,
     w3a16_gemm_route,
 )
 
@@ -47,5 +48,6 @@ __all__ = [
     "w3a16_gemm",
     "w3a16_gemm_native",
     "w3a16_gemm_noalloc",
+    "w3a16_gemm_launches",
     "w3a16_gemm_route",
 ]

@@ -49,6 +49,7 @@ SIGNATURES = [
     ("w3_packed_from_native", ctypes.c_int, [_P, _P, _I64, _I64, _P]),
     ("w3a16_gemm_native", ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P]),
     ("w3a16_gemm_route", ctypes.c_char_p, [_I64, _I64, _I64, ctypes.c_int32]),
+    ("w3a16_gemm_launches", ctypes.c_int32, [_I64, _I64, _I64, ctypes.c_int32]),
     ("w3_check_device_error", ctypes.c_int, [_P]),
 ]
 
@@ -285,6 +286,17 @@ def w3a16_gemm_route(M: int, N: int, K: int, num_sms: int | None = None) -> str:
     if r is None:
         raise ValueError(f"w3a16_gemm_route: no route for M={M} N={N} K={K} num_sms={num_sms}")
     return r.decode()
+
+
+def w3a16_gemm_launches(M: int, N: int, K: int, num_sms: int | None = None) -> int:
+    """How many kernels one w3a16_gemm call launches for M x N x K (see include/w3a16.h).
+    num_sms defaults to the current CUDA device's SM count."""
+    if num_sms is None:
+        num_sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    n = lib().w3a16_gemm_launches(M, N, K, num_sms)
+    if n < 0:
+        raise ValueError(f"w3a16_gemm_launches: no route for M={M} N={N} K={K} num_sms={num_sms}")
+    return n
 
 
 def w3_check_device_error(stream=None) -> None:

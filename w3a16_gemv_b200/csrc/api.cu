@@ -625,6 +625,17 @@ Route choose_route(int64_t M, int64_t N, int64_t K, int sms) {
     return Route::Passes;
 }
 
+// Kernels one w3a16_gemm call launches for M x N x K: the route's main kernel, plus the
+// fix-up kernel where the tensor-core decode splits a tile between CTAs; the passes route
+// adds up its 16-row passes (one kernel each).
+int64_t launches_for(int64_t M, int64_t N, int64_t K, int sms) {
+    switch (choose_route(M, N, K, sms)) {
+        case Route::DecodeTc32: return decode_tc32::plan(N, K, sms).P > 1 ? 2 : 1;
+        case Route::Passes: return (M + 15) / 16;
+        default: return 1;
+    }
+}
+
 const char *route_name(Route r) {
     switch (r) {
         case Route::DecodeSplit: return "decode_split";
@@ -944,6 +955,12 @@ w3_status w3a16_gemm_native(const uint16_t *x, const int32_t *native, const uint
 const char *w3a16_gemm_route(int64_t M, int64_t N, int64_t K, int32_t num_sms) {
     if (M < 1 || check_nk(N, K) != W3_OK || M > kMaxDim || num_sms < 1) return nullptr;
     return route_name(choose_route(M, N, K, num_sms));
+}
+
+int32_t w3a16_gemm_launches(int64_t M, int64_t N, int64_t K, int32_t num_sms) {
+    if (M < 1 || check_nk(N, K) != W3_OK || M > kMaxDim || num_sms < 1) return -1;
+    const int64_t n = launches_for(M, N, K, num_sms);
+    return n > INT32_MAX ? INT32_MAX : static_cast<int32_t>(n);
 }
 
 #ifdef W3_TEST_HOOKS
