@@ -39,6 +39,12 @@ MUTANTS = [
     ("native_row_stride_4", "int64_t row = 32 * b + l / 4 + 8 * h;", "int64_t row = 32 * b + l / 4 + 4 * h;", 2),
     ("native_words_of_lane_block", "int64_t word = 12 * g + 3 * (l % 4) + i;",
      "int64_t word = 12 * g + 3 * (l / 8) + i;", 2),
+    # the row norms that scale every parity tolerance: a wrong norm would loosen the GPU tests
+    ("norm_without_sqrt", "out[n] = sqrt(ss);", "out[n] = ss;", 1),
+    ("norm_of_first_group_only", "for (int64_t k = 0; k < K; ++k) ss +=", "for (int64_t k = 0; k < 128; ++k) ss +=", 1),
+    # the multi-threaded product (the full-size parity tests use it) dropping its last output row
+    ("threads_skip_last_row", "        for (int64_t n = 0; n < N; ++n) {\n            if (!wrow) continue;",
+     "        for (int64_t n = 0; n < N - 1; ++n) {\n            if (!wrow) continue;", 1),
 ]
 
 
